@@ -1,0 +1,184 @@
+// api.cu — host side of libfa.so: argument validation, TMA descriptor encoding,
+// launch configuration and the extern "C" entry points declared in include/fa.h.
+//
+// The whole library is one translation unit (this file includes the kernel
+// headers), so the device status word and the kernels live together.
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/fa.h"
+#include "sm100.cuh"
+#include "fwd.cuh"
+#include "bwd.cuh"
+
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+
+int cuda_fail(cudaError_t e) {
+  t_last_cuda_error = static_cast<int>(e);
+  return FA_ERR_CUDA;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// [B*H, N, d] row-major tensor seen as a 3-D TMA tensor (d, N, B*H); box of
+// 128 bytes x 128 rows with the 128-byte swizzle.  Rows beyond N read as zero.
+int encode_qkv_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, int d, int N, int BH,
+                   CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
+  auto fn = encode_fn();
+  if (!fn) return cuda_fail(cudaErrorNotSupported);
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * elem_bytes,
+                           static_cast<cuuint64_t>(d) * static_cast<cuuint64_t>(N) * elem_bytes};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem_bytes), 128, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+  return FA_OK;
+}
+
+int check_common(const void* q, const void* k, const void* v, const void* o, const void* lse, int B, int H, int N,
+                 int d, float scale) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const long long total = static_cast<long long>(B) * H * N * d;
+  if (total >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGNMENT;
+  return FA_OK;
+}
+
+template <typename T, int D, bool FP8P>
+int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int causal,
+               float scale, float S, int kv_order, unsigned long long* stats, int n_sink, cudaStream_t stream) {
+  using C = fa::FwdCfg<T, D, FP8P>;
+  constexpr CUtensorMapDataType dt =
+      sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  const int BH = B * H;
+  CUtensorMap mq, mk, mv;
+  int st;
+  if ((st = encode_qkv_map(&mq, q, dt, sizeof(T), D, N, BH)) != FA_OK) return st;
+  if ((st = encode_qkv_map(&mk, k, dt, sizeof(T), D, N, BH)) != FA_OK) return st;
+  // fp32 V feeds the tf32 MMA as an MN-major operand, which needs the 32-byte-atom swizzle
+  if ((st = encode_qkv_map(&mv, v, dt, sizeof(T), D, N, BH,
+                           sizeof(T) == 2 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B)) != FA_OK)
+    return st;
+  fa::FwdArgs a;
+  a.o = o;
+  a.lse = lse;
+  a.N = N;
+  a.BH = BH;
+  a.nblk = (N + 255) / 256;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.p_scale = S;
+  a.causal = causal ? 1 : 0;
+  a.kv_order = kv_order;
+  a.stats = stats;
+  a.n_sink = n_sink;
+  auto kern = fa::fa_fwd_kernel<T, D, FP8P>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const long long grid = static_cast<long long>(a.nblk) * BH;
+  kern<<<static_cast<unsigned>(grid), C::NTHREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d, int causal,
+           float scale, void* stream) {
+  int st = check_common(q, k, v, o, lse, B, H, N, d, scale);
+  if (st != FA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 64) return launch_fwd<__nv_bfloat16, 64, false>(q, k, v, o, lse, B, H, N, causal, scale, 1.f, 0, nullptr, 0, s);
+  return launch_fwd<__nv_bfloat16, 128, false>(q, k, v, o, lse, B, H, N, causal, scale, 1.f, 0, nullptr, 0, s);
+}
+
+int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int H, int N, int d,
+               int causal, float scale, void* stream) {
+  int st = check_common(q, k, v, o, lse, B, H, N, d, scale);
+  if (st != FA_OK) return st;
+  if (d != 64) return FA_ERR_UNSUPPORTED;  // fp32 tiles of 128 x 128 do not fit the shared-memory ring
+  return launch_fwd<float, 64, false>(q, k, v, o, lse, B, H, N, causal, scale, 1.f, 0, nullptr, 0,
+                                      static_cast<cudaStream_t>(stream));
+}
+
+int fa_fwd_fp8p(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                int causal, float scale, float S, int kv_order, unsigned long long* stats, int n_sink,
+                void* stream) {
+  int st = check_common(q, k, v, o, lse, B, H, N, d, scale);
+  if (st != FA_OK) return st;
+  if (!(std::isfinite(S) && S > 0.f)) return FA_ERR_INVALID_ARG;
+  if (kv_order != 0 && kv_order != 1) return FA_ERR_INVALID_ARG;
+  if (n_sink < 0) return FA_ERR_INVALID_ARG;
+  if (stats && (reinterpret_cast<uintptr_t>(stats) & 7u)) return FA_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 64)
+    return launch_fwd<__nv_bfloat16, 64, true>(q, k, v, o, lse, B, H, N, causal, scale, S, kv_order, stats, n_sink, s);
+  return launch_fwd<__nv_bfloat16, 128, true>(q, k, v, o, lse, B, H, N, causal, scale, S, kv_order, stats, n_sink, s);
+}
+
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
+  (void)B; (void)H; (void)N; (void)d;
+  return 0;
+}
+
+int fa_bwd(const void*, const void*, const void*, const void*, const void*, const float*, void*, void*, void*, int,
+           int, int, int, int, float, void*, size_t, void*) {
+  return FA_ERR_UNSUPPORTED;
+}
+
+const char* fa_status_string(int status) {
+  switch (status & 0xFF) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_ALIGNMENT: return "FA_ERR_ALIGNMENT";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    default: return "FA_ERR_UNKNOWN";
+  }
+}
+
+int fa_last_cuda_error(void) { return t_last_cuda_error; }
+
+int fa_check_status(void) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e);
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, fa::g_fa_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(fa::g_fa_status, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return v & 0xFF;
+}
+
+}  // extern "C"

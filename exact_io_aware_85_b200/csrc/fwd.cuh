@@ -1,0 +1,476 @@
+// fwd.cuh — exact attention forward on B200: TMA + tcgen05 + TMEM, warp-specialised.
+//
+// Algorithm ("flash-attention-trading-models", sections "El algoritmo de atencion
+// flash" and "La recurrencia de softmax en linea"; "FlashAttention (IT)", "Tiling",
+// "Calcolo online del Softmax", "Fusione delle operazioni"): split Q into row tiles
+// of 128 and K, V into column tiles of 128; for each Q tile visit the K/V tiles,
+// keep the running row max m and running sum l, rescale the partial O when m grows,
+// never write S or P to device memory, and normalise O once at the end (the
+// deferred rescale of FlashAttention-2, same page, section "FA2").
+//
+// One CTA owns two Q tiles (256 query rows) of one (batch, head) and runs on its
+// own SM.  Warp roles (FlashAttention-3's producer/consumer split, same page,
+// section "FA3", re-cast for tcgen05):
+//   warps 0-3  softmax for Q tile 0   (thread r owns row r = TMEM lane r)
+//   warps 4-7  softmax for Q tile 1
+//   warp  8    TMA producer: Q0, Q1 once, then K_j and V_j through a ring
+//   warp  9    tcgen05.mma issuer (one thread) and TMEM owner
+// Tensor memory (512 columns x 128 lanes, fp32):
+//   [0,128)   S0 = Q0 K_j^T   (P0 is written over its first columns as bf16)
+//   [128,256) S1 = Q1 K_j^T   (P1 likewise)
+//   [256,256+D) O0, then O1   (fp32 accumulators)
+// The MMA thread interleaves the two tiles so that the tensor core works on one
+// tile while the softmax warps work on the other (FA3 "interleaved matmul and
+// softmax"):  S0(j+1) is issued right after PV0(j), before waiting for P1(j).
+// Every tcgen05.commit covers all earlier MMAs of the thread, so the arrival of
+// "S_i(j) ready" also means "PV_i(j-1) done": the softmax warps may then rescale
+// O_i in TMEM before handing P_i(j) back.
+//
+// Causal masking ("flash-attention-trading-models", section on causal masking):
+// key tiles wholly in the future of a Q tile are never loaded or multiplied;
+// the diagonal tile and the ragged last key tile are masked element-wise.
+#pragma once
+#include "sm100.cuh"
+
+namespace fa {
+
+template <typename T>
+struct ElemTraits;
+template <>
+struct ElemTraits<__nv_bfloat16> {
+  static constexpr int kBytes = 2;
+  static constexpr uint32_t kFmt = kFmtBF16;
+};
+template <>
+struct ElemTraits<float> {
+  static constexpr int kBytes = 4;
+  static constexpr uint32_t kFmt = kFmtTF32;
+};
+
+struct FwdArgs {
+  void* o;
+  float* lse;
+  int N;          // sequence length
+  int BH;         // batch * heads
+  int nblk;       // ceil(N / 256): CTAs per (batch, head)
+  float scale_log2;  // softmax scale * log2(e)
+  float p_scale;     // static scale S of the E4M3 P-cast (1 otherwise)
+  int causal;
+  int kv_order;      // 0: key tiles 0..T-1, 1: T-1..0
+  unsigned long long* stats;
+  int n_sink;
+};
+
+template <typename T, int D, bool FP8P>
+struct FwdCfg {
+  static constexpr int EB = ElemTraits<T>::kBytes;
+  static constexpr int BOX_COLS = 128 / EB;            // elements in one 128-byte swizzled row
+  static constexpr int NBOX = D / BOX_COLS;            // TMA boxes across the head dim
+  static constexpr int BOX_BYTES = 128 * 128;          // 128 rows x 128 bytes
+  static constexpr int TILE_BYTES = NBOX * BOX_BYTES;  // one 128 x D tile
+  static constexpr int KSTEP = 32 / EB;                // K elements per MMA (32 bytes)
+  static constexpr int KSTEPS_PER_BOX = BOX_COLS / KSTEP;
+  static constexpr int NK_QK = D / KSTEP;              // MMAs for one S tile
+  static constexpr int NK_PV = 128 / KSTEP;            // MMAs for one PV tile
+  static constexpr int NSTAGE = (TILE_BYTES <= 16384) ? 3 : 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = 2 * TILE_BYTES;
+  static constexpr int OFF_V = OFF_K + NSTAGE * TILE_BYTES;
+  static constexpr int SMEM_BYTES = OFF_V + NSTAGE * TILE_BYTES + 1024;  // + alignment slack
+  static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
+  static constexpr int NTHREADS = 320;
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+  static_assert(COL_O1 + D <= 512, "tensor memory budget");
+};
+
+template <typename T, int D, bool FP8P>
+__global__ void __launch_bounds__(320, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
+  using C = FwdCfg<T, D, FP8P>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ uint64_t bar_q, bar_kf[C::NSTAGE], bar_ke[C::NSTAGE], bar_vf[C::NSTAGE], bar_ve[C::NSTAGE];
+  __shared__ uint64_t bar_s[2], bar_p[2], bar_o[2], bar_done;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- work decode: heaviest query blocks first when causal -----------------
+  const int N = a.N;
+  const int bh = blockIdx.x % a.BH;
+  int qblk = blockIdx.x / a.BH;
+  if (a.causal) qblk = a.nblk - 1 - qblk;
+  const int m0 = qblk * 256;
+  const int n_kv = (N + 127) >> 7;
+  const int qt0 = m0 >> 7;
+  const bool valid0 = m0 < N, valid1 = m0 + 128 < N;
+  const int kv_end0 = valid0 ? (a.causal ? min(n_kv, qt0 + 1) : n_kv) : 0;
+  const int kv_end1 = valid1 ? (a.causal ? min(n_kv, qt0 + 2) : n_kv) : 0;
+  const int n_steps = max(kv_end0, kv_end1);
+  const int rev = a.kv_order;
+
+  // ---- setup ---------------------------------------------------------------
+  if (warp == 9) {
+    tmem_alloc(&tmem_base_sh, 512);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    abort_sh = 0;
+    mbar_init(&bar_q, 1);
+    for (int s = 0; s < C::NSTAGE; ++s) {
+      mbar_init(&bar_kf[s], 1);
+      mbar_init(&bar_ke[s], 1);
+      mbar_init(&bar_vf[s], 1);
+      mbar_init(&bar_ve[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_s[i], 1);
+      mbar_init(&bar_p[i], 128);
+      mbar_init(&bar_o[i], 1);
+    }
+    mbar_init(&bar_done, 1);
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp == 8) {
+    // ======================= TMA producer ===================================
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      mbar_arrive_expect_tx(&bar_q, (valid1 ? 2 : 1) * C::TILE_BYTES);
+      for (int b = 0; b < C::NBOX; ++b) {
+        tma_load_3d(smem + C::OFF_Q + b * C::BOX_BYTES, &tmQ, &bar_q, b * C::BOX_COLS, m0, bh);
+        if (valid1)
+          tma_load_3d(smem + C::OFF_Q + C::TILE_BYTES + b * C::BOX_BYTES, &tmQ, &bar_q, b * C::BOX_COLS, m0 + 128,
+                      bh);
+      }
+      for (int t = 0; t < n_steps; ++t) {
+        const int j = rev ? n_steps - 1 - t : t;
+        const int s = t % C::NSTAGE;
+        const uint32_t ph = (t / C::NSTAGE) & 1;
+        if (!mbar_wait(&bar_ke[s], ph ^ 1, &abort_sh, 1)) break;
+        mbar_arrive_expect_tx(&bar_kf[s], C::TILE_BYTES);
+        for (int b = 0; b < C::NBOX; ++b)
+          tma_load_3d(smem + C::OFF_K + s * C::TILE_BYTES + b * C::BOX_BYTES, &tmK, &bar_kf[s], b * C::BOX_COLS,
+                      j * 128, bh);
+        if (!mbar_wait(&bar_ve[s], ph ^ 1, &abort_sh, 2)) break;
+        mbar_arrive_expect_tx(&bar_vf[s], C::TILE_BYTES);
+        for (int b = 0; b < C::NBOX; ++b)
+          tma_load_3d(smem + C::OFF_V + s * C::TILE_BYTES + b * C::BOX_BYTES, &tmV, &bar_vf[s], b * C::BOX_COLS,
+                      j * 128, bh);
+      }
+      // teardown: let every issued copy land before the CTA can exit
+      const int first = max(0, n_steps - C::NSTAGE);
+      for (int t = first; t < n_steps; ++t) {
+        const int s = t % C::NSTAGE;
+        const uint32_t ph = (t / C::NSTAGE) & 1;
+        mbar_wait_drain(&bar_kf[s], ph, 100000000ull);
+        mbar_wait_drain(&bar_vf[s], ph, 100000000ull);
+      }
+    }
+  } else if (warp == 9) {
+    // ======================= tcgen05.mma issuer =============================
+    // The whole warp follows the control flow (the fp32 path uses all lanes to
+    // round operand tiles); lane 0 alone issues MMAs and commits.
+    {
+      const bool leader = lane == 0;
+      // every lane waits (each gets the acquire), then the warp agrees on the outcome
+      auto warp_wait = [&](uint64_t* bar, uint32_t parity, volatile int* ab, int site) {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, ab, site));
+      };
+      constexpr uint32_t idesc_s = make_idesc(128, 128, ElemTraits<T>::kFmt, 0, 0);
+      constexpr uint32_t idesc_pv = make_idesc(128, D, ElemTraits<T>::kFmt, 0, 1);
+      const uint32_t q_addr = smem_u32(smem + C::OFF_Q);
+      const uint32_t k_addr = smem_u32(smem + C::OFF_K);
+      const uint32_t v_addr = smem_u32(smem + C::OFF_V);
+      int pv_count[2] = {0, 0};
+      const int kv_end[2] = {kv_end0, kv_end1};
+
+      auto issue_s = [&](int i, int s) {
+        const uint32_t qa = q_addr + i * C::TILE_BYTES;
+        const uint32_t ka = k_addr + s * C::TILE_BYTES;
+#pragma unroll
+        for (int k = 0; k < C::NK_QK; ++k) {
+          const uint32_t off = (k / C::KSTEPS_PER_BOX) * C::BOX_BYTES + (k % C::KSTEPS_PER_BOX) * 32;
+          const uint64_t ad = make_sdesc_sw128(qa + off, 16, 1024);
+          const uint64_t bd = make_sdesc_sw128(ka + off, 16, 1024);
+          if (!leader) continue;
+          if constexpr (C::EB == 2)
+            mma_ss(tmem + (i ? C::COL_S1 : C::COL_S0), ad, bd, idesc_s, k > 0);
+          else
+            mma_ss_tf32(tmem + (i ? C::COL_S1 : C::COL_S0), ad, bd, idesc_s, k > 0);
+        }
+        if (leader) mma_commit(&bar_s[i]);
+      };
+      auto issue_pv = [&](int i, int s) {
+        const uint32_t va = v_addr + s * C::TILE_BYTES;
+        const uint32_t pcol = tmem + (i ? C::COL_S1 : C::COL_S0);
+        const uint32_t ocol = tmem + (i ? C::COL_O1 : C::COL_O0);
+#pragma unroll
+        for (int k = 0; k < C::NK_PV; ++k) {
+          // V is the MN-major B operand: 128B swizzle (bf16) or the 32-byte-atom
+          // 128B swizzle (tf32, whose only MN-major layout), K rows 128 B apart.
+          const uint64_t bd = C::EB == 2 ? make_sdesc_sw128(va + k * C::KSTEP * 128, C::BOX_BYTES, 1024)
+                                         : make_sdesc_sw128_32b(va + k * C::KSTEP * 128, C::BOX_BYTES, 512);
+          const uint32_t acc = (pv_count[i] > 0 || k > 0) ? 1u : 0u;
+          if (!leader) continue;
+          if constexpr (C::EB == 2)
+            mma_ts(ocol, pcol + k * 8, bd, idesc_pv, acc);
+          else
+            mma_ts_tf32(ocol, pcol + k * 8, bd, idesc_pv, acc);
+        }
+        pv_count[i]++;
+        if (leader && pv_count[i] == kv_end[i]) mma_commit(&bar_o[i]);
+      };
+      // fp32 inputs: the tensor core reads the top 19 bits of each operand
+      // (truncation); Q and K are rounded to tf32 to nearest-even in place first,
+      // so that the scores, and with them the logsumexp, carry no truncation bias.
+      auto round_tile_tf32 = [&](uint32_t byte_off, int nbytes) {
+        if constexpr (C::EB == 4) {
+          uint4* p = reinterpret_cast<uint4*>(smem + byte_off);
+          for (int idx = lane; idx < nbytes / 16; idx += 32) {
+            uint4 w = p[idx];
+            w.x = (w.x + 0xFFFu + ((w.x >> 13) & 1u)) & 0xFFFFE000u;
+            w.y = (w.y + 0xFFFu + ((w.y >> 13) & 1u)) & 0xFFFFE000u;
+            w.z = (w.z + 0xFFFu + ((w.z >> 13) & 1u)) & 0xFFFFE000u;
+            w.w = (w.w + 0xFFFu + ((w.w >> 13) & 1u)) & 0xFFFFE000u;
+            p[idx] = w;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+      };
+
+      bool ok = warp_wait(&bar_q, 0, &abort_sh, 3);
+      if (ok) round_tile_tf32(C::OFF_Q, (valid1 ? 2 : 1) * C::TILE_BYTES);
+      if (ok && n_steps > 0) {
+        const int j0 = rev ? n_steps - 1 : 0;
+        ok = warp_wait(&bar_kf[0], 0, &abort_sh, 4);
+        if (ok) {
+          round_tile_tf32(C::OFF_K, C::TILE_BYTES);
+          tc_fence_after();
+          if (j0 < kv_end0) issue_s(0, 0);
+          if (j0 < kv_end1) issue_s(1, 0);
+          if (leader) mma_commit(&bar_ke[0]);
+        }
+      }
+      for (int t = 0; ok && t < n_steps; ++t) {
+        const int j = rev ? n_steps - 1 - t : t;
+        const int s = t % C::NSTAGE;
+        const uint32_t ph = (t / C::NSTAGE) & 1;
+        const bool has_next = t + 1 < n_steps;
+        const int jn = rev ? n_steps - 2 - t : t + 1;
+        const int sn = (t + 1) % C::NSTAGE;
+        const uint32_t phn = ((t + 1) / C::NSTAGE) & 1;
+        bool kn_ready = false;
+        if (!(ok = warp_wait(&bar_vf[s], ph, &abort_sh, 5))) break;
+        if (j < kv_end0) {
+          if (!(ok = warp_wait(&bar_p[0], pv_count[0] & 1, &abort_sh, 6))) break;
+          tc_fence_after();
+          issue_pv(0, s);
+        }
+        if (has_next && jn < kv_end0) {
+          if (!(ok = warp_wait(&bar_kf[sn], phn, &abort_sh, 7))) break;
+          kn_ready = true;
+          round_tile_tf32(C::OFF_K + sn * C::TILE_BYTES, C::TILE_BYTES);
+          tc_fence_after();
+          issue_s(0, sn);
+        }
+        if (j < kv_end1) {
+          if (!(ok = warp_wait(&bar_p[1], pv_count[1] & 1, &abort_sh, 8))) break;
+          tc_fence_after();
+          issue_pv(1, s);
+        }
+        if (leader) mma_commit(&bar_ve[s]);
+        if (has_next) {
+          if (jn < kv_end1) {
+            if (!kn_ready) {
+              if (!(ok = warp_wait(&bar_kf[sn], phn, &abort_sh, 9))) break;
+              round_tile_tf32(C::OFF_K + sn * C::TILE_BYTES, C::TILE_BYTES);
+              tc_fence_after();
+            }
+            issue_s(1, sn);
+          }
+          if (leader) mma_commit(&bar_ke[sn]);
+        }
+      }
+      // teardown: every MMA of this thread must be finished before TMEM is freed
+      if (leader) {
+        mma_commit(&bar_done);
+        mbar_wait_drain(&bar_done, 0, 100000000ull);
+      }
+      __syncwarp();
+    }
+  } else {
+    // ======================= softmax warpgroups =============================
+    const int i = warp >> 2;                       // Q tile
+    const int r = threadIdx.x & 127;               // row in tile == TMEM lane
+    const int row = m0 + 128 * i + r;              // query index
+    const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    const uint32_t tS = tmem + lane_base + (i ? C::COL_S1 : C::COL_S0);
+    const uint32_t tO = tmem + lane_base + (i ? C::COL_O1 : C::COL_O0);
+    const int kv_end = i ? kv_end1 : kv_end0;
+    const int qt = qt0 + i;
+    const float c = a.scale_log2;
+    float m_run = -INFINITY, l_run = 0.f;
+    uint32_t fl_sink = 0, fl_non = 0;
+    int cnt = 0;
+    bool ok = true;
+    if (kv_end > 0) {
+      for (int t = 0; t < n_steps; ++t) {
+        const int j = rev ? n_steps - 1 - t : t;
+        if (j >= kv_end) continue;
+        if (!(ok = mbar_wait(&bar_s[i], cnt & 1, &abort_sh, 10 + i))) break;
+        tc_fence_after();
+        float sv[128];
+        tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
+        tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+        tmem_wait_ld();
+        const int kbase = j * 128;
+        if (kbase + 128 > N || (a.causal && j == qt)) {
+          const int lim = a.causal ? min(N - 1, row) : N - 1;  // last admissible key
+#pragma unroll
+          for (int cc = 0; cc < 128; ++cc)
+            if (kbase + cc > lim) sv[cc] = -INFINITY;
+        }
+        float mx = sv[0];
+#pragma unroll
+        for (int cc = 1; cc < 128; ++cc) mx = fmaxf(mx, sv[cc]);
+        float m_new = fmaxf(m_run, mx * c);
+        // Lazy rescale: keep the old max while the growth stays within 2^8 (exps stay
+        // <= 256, safe in bf16/fp32).  The FP8 P-cast needs the exact running max.
+        if (!FP8P && m_new - m_run <= 8.0f) m_new = m_run;
+        const float alpha = ex2_approx(m_run - m_new);
+        if (cnt > 0 && __any_sync(0xffffffffu, m_new != m_run)) {
+#pragma unroll
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t ov[32];
+            tmem_ld32(tO + ch * 32, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            tmem_st32(tO + ch * 32, ov);
+          }
+        }
+        l_run *= alpha;
+        m_run = m_new;
+        const float neg_m = -m_run;
+        float rs = 0.f;
+        if constexpr (C::EB == 2) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t pk[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float p0 = ex2_approx(fmaf(sv[h * 64 + 2 * e], c, neg_m));
+              const float p1 = ex2_approx(fmaf(sv[h * 64 + 2 * e + 1], c, neg_m));
+              rs += p0 + p1;
+              if constexpr (FP8P) {
+                float q0, q1;
+                pk[e] = e4m3_roundtrip_bf16x2(p0 * a.p_scale, p1 * a.p_scale, q0, q1);
+                if (a.stats != nullptr && row < N) {
+                  const int k0 = kbase + h * 64 + 2 * e;
+                  const int lim = a.causal ? min(N - 1, row) : N - 1;
+                  if (k0 <= lim && q0 == 0.f) { if (k0 < a.n_sink) ++fl_sink; else ++fl_non; }
+                  if (k0 + 1 <= lim && q1 == 0.f) { if (k0 + 1 < a.n_sink) ++fl_sink; else ++fl_non; }
+                }
+              } else {
+                pk[e] = pack_bf16x2(p0, p1);
+              }
+            }
+            tmem_st32(tS + h * 32, pk);
+          }
+        } else {
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            uint32_t pk[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float p = ex2_approx(fmaf(sv[h * 32 + e], c, neg_m));
+              rs += p;
+              pk[e] = __float_as_uint(p);
+            }
+            tmem_st32(tS + h * 32, pk);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bar_p[i]);
+        l_run += rs;
+        ++cnt;
+      }
+      // ---- epilogue: O / l -> global, LSE -> global --------------------------
+      if (ok) ok = mbar_wait(&bar_o[i], 0, &abort_sh, 12 + i);
+      if (ok) {
+        tc_fence_after();
+        const float inv = 1.0f / (l_run * a.p_scale);
+        T* orow = reinterpret_cast<T*>(a.o) + (static_cast<size_t>(bh) * N + row) * D;
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t ov[32];
+          tmem_ld32(tO + ch * 32, ov);
+          tmem_wait_ld();
+          if (row < N) {
+            if constexpr (C::EB == 2) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+              for (int v4 = 0; v4 < 4; ++v4) {
+                uint4 w;
+                w.x = pack_bf16x2(__uint_as_float(ov[8 * v4 + 0]) * inv, __uint_as_float(ov[8 * v4 + 1]) * inv);
+                w.y = pack_bf16x2(__uint_as_float(ov[8 * v4 + 2]) * inv, __uint_as_float(ov[8 * v4 + 3]) * inv);
+                w.z = pack_bf16x2(__uint_as_float(ov[8 * v4 + 4]) * inv, __uint_as_float(ov[8 * v4 + 5]) * inv);
+                w.w = pack_bf16x2(__uint_as_float(ov[8 * v4 + 6]) * inv, __uint_as_float(ov[8 * v4 + 7]) * inv);
+                dst[v4] = w;
+              }
+            } else {
+              float4* dst = reinterpret_cast<float4*>(orow + ch * 32);
+#pragma unroll
+              for (int v4 = 0; v4 < 8; ++v4)
+                dst[v4] = make_float4(__uint_as_float(ov[4 * v4 + 0]) * inv, __uint_as_float(ov[4 * v4 + 1]) * inv,
+                                      __uint_as_float(ov[4 * v4 + 2]) * inv, __uint_as_float(ov[4 * v4 + 3]) * inv);
+            }
+          }
+        }
+        if (row < N) a.lse[static_cast<size_t>(bh) * N + row] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
+      }
+      if constexpr (FP8P) {
+        if (a.stats != nullptr) {
+          // totals are exact counts of admissible keys for this row
+          uint32_t nk = 0;
+          if (row < N) nk = a.causal ? static_cast<uint32_t>(row + 1) : static_cast<uint32_t>(N);
+          const uint32_t ts = min(nk, static_cast<uint32_t>(max(a.n_sink, 0)));
+          const uint32_t tn = nk - ts;
+          const uint32_t v0 = __reduce_add_sync(0xffffffffu, fl_sink);
+          const uint32_t v1 = __reduce_add_sync(0xffffffffu, ts);
+          const uint32_t v2 = __reduce_add_sync(0xffffffffu, fl_non);
+          const uint32_t v3 = __reduce_add_sync(0xffffffffu, tn);
+          if (lane == 0) {
+            atomicAdd(a.stats + 0, static_cast<unsigned long long>(v0));
+            atomicAdd(a.stats + 1, static_cast<unsigned long long>(v1));
+            atomicAdd(a.stats + 2, static_cast<unsigned long long>(v2));
+            atomicAdd(a.stats + 3, static_cast<unsigned long long>(v3));
+          }
+        }
+      }
+    }
+  }
+
+  // ---- teardown ------------------------------------------------------------
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fa

@@ -1,0 +1,106 @@
+"""ctypes binding of libfa.so with the entry-point names of include/fa.h.
+
+Argument marshalling only: sizes and raw device pointers are taken from torch
+tensors (torch is the allocator and stream owner), every step of the
+computation runs in the library's CUDA kernels.  There is no fallback: if the
+library is missing the import fails, and a non-zero status raises FAError.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"libfa.so is not built ({_LIB_PATH}); run `python -m exact_io_aware_85_b200.build`")
+
+lib = ctypes.CDLL(_LIB_PATH)
+_vp, _ci, _cf, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+lib.fa_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _cf, _vp]
+lib.fa_fwd_f32.argtypes = [_vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _cf, _vp]
+lib.fa_fwd_fp8p.argtypes = [_vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _cf, _cf, _ci, _vp, _ci, _vp]
+lib.fa_bwd_workspace_bytes.restype = _sz
+lib.fa_bwd_workspace_bytes.argtypes = [_ci, _ci, _ci, _ci]
+lib.fa_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _cf, _vp, _sz, _vp]
+lib.fa_status_string.restype = ctypes.c_char_p
+lib.fa_status_string.argtypes = [_ci]
+lib.fa_last_cuda_error.restype = _ci
+lib.fa_check_status.restype = _ci
+
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_ALIGNMENT, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(6)
+EXPORTS = ("fa_fwd", "fa_fwd_f32", "fa_fwd_fp8p", "fa_bwd_workspace_bytes", "fa_bwd", "fa_status_string",
+           "fa_last_cuda_error", "fa_check_status")
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib.fa_status_string(status).decode()
+        if status == FA_ERR_CUDA:
+            msg += f" (cudaError {lib.fa_last_cuda_error()})"
+        super().__init__(f"{where}: {msg}")
+
+
+def _check(status: int, where: str) -> None:
+    if status != FA_OK:
+        raise FAError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dims(q):
+    if q.dim() != 4:
+        raise ValueError("expected [B, H, N, d] tensors")
+    return tuple(int(x) for x in q.shape)
+
+
+def fa_fwd(q, k, v, o, lse, causal: bool, scale: float, stream=None) -> None:
+    """bf16 forward: writes o (bf16 [B,H,N,d]) and lse (fp32 [B,H,N])."""
+    B, H, N, d = _dims(q)
+    _check(lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, int(causal), float(scale),
+                      _stream(stream)), "fa_fwd")
+
+
+def fa_fwd_f32(q, k, v, o, lse, causal: bool, scale: float, stream=None) -> None:
+    """fp32 forward on the tf32 tensor-core path."""
+    B, H, N, d = _dims(q)
+    _check(lib.fa_fwd_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, int(causal), float(scale),
+                          _stream(stream)), "fa_fwd_f32")
+
+
+def fa_fwd_fp8p(q, k, v, o, lse, causal: bool, scale: float, S: float, kv_order: int, stats=None, n_sink: int = 4,
+                stream=None) -> None:
+    """Forward with P cast to E4M3 under static scale S; stats (uint64 [4] as int64) is added to."""
+    B, H, N, d = _dims(q)
+    _check(lib.fa_fwd_fp8p(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, int(causal), float(scale),
+                           float(S), int(kv_order), _ptr(stats), int(n_sink), _stream(stream)), "fa_fwd_fp8p")
+
+
+def fa_bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(lib.fa_bwd_workspace_bytes(B, H, N, d))
+
+
+def fa_bwd(q, k, v, o, do, lse, dq, dk, dv, causal: bool, scale: float, workspace, stream=None) -> None:
+    """Backward: writes dq, dk, dv (bf16 [B,H,N,d]); workspace is a uint8 device tensor."""
+    B, H, N, d = _dims(q)
+    _check(lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), B, H,
+                      N, d, int(causal), float(scale), _ptr(workspace), int(workspace.numel()),
+                      _stream(stream)), "fa_bwd")
+
+
+def fa_status_string(status: int) -> str:
+    return lib.fa_status_string(int(status)).decode()
+
+
+def fa_check_status() -> int:
+    return int(lib.fa_check_status())

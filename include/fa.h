@@ -1,0 +1,106 @@
+/*
+ * fa.h -- C ABI of libfa.so: exact IO-aware tiled attention on NVIDIA B200 (sm_100a).
+ *
+ * The operation is O = softmax(scale * Q K^T) V, computed tile by tile with the
+ * online-softmax recurrence so that the N x N score matrix never reaches device
+ * memory ("flash-attention-trading-models", sections "El algoritmo de atencion
+ * flash" and "La recurrencia de softmax en linea"; "FlashAttention (IT)",
+ * sections "Tiling" and "Calcolo online del Softmax").  Alongside O every entry
+ * point writes the per-row logsumexp, the O(N) statistic that the backward pass
+ * needs ("flash-attention-trading-models", section "Pase hacia atras").
+ *
+ * Conventions shared by every entry point
+ *  - Layout: q, k, v, o, dO, dq, dk, dv are contiguous row-major [B, H, N, d]
+ *    device arrays (the (batch, heads, seq, head_dim) layout of the pages'
+ *    framework example); lse is a contiguous [B, H, N] float32 device array.
+ *    LSE is the natural-log logsumexp of the scaled scores of each query row.
+ *  - Sizes: B >= 1, H >= 1, N >= 1, d in {64, 128}; B*H*N*d < 2^31.
+ *  - scale: the softmax scale (usually 1/sqrt(d)); finite and > 0.
+ *  - causal != 0: query i attends to keys j <= i (square, top-left aligned);
+ *    tiles that lie entirely in the future are skipped, never loaded.
+ *  - Alignment: every device pointer 16-byte aligned.
+ *  - Ownership: the caller allocates and owns every buffer.  The library never
+ *    allocates, frees or synchronises (fa_check_status excepted); all work is
+ *    enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream).
+ *  - Errors: invalid arguments are rejected before anything is launched and
+ *    return a non-zero fa_status; there is no fallback path.  A failed launch
+ *    returns FA_ERR_CUDA (fa_last_cuda_error() gives the cudaError_t).  Device
+ *    pipelines that stall past a bound record FA_ERR_TIMEOUT in a device status
+ *    word that fa_check_status() reads after the caller's work has finished.
+ *  - Thread safety: entry points may be called concurrently from host threads.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, bad scale/S/kv_order */
+  FA_ERR_UNSUPPORTED = 2, /* head dim other than 64/128, or sizes over the limits */
+  FA_ERR_ALIGNMENT = 3,   /* a pointer that is not 16-byte aligned */
+  FA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed */
+  FA_ERR_TIMEOUT = 5      /* a device-side wait gave up (reported by fa_check_status) */
+} fa_status;
+
+/* Forward, bf16 in/out, fp32 accumulation on the tensor cores.
+ * q, k, v: bf16 [B,H,N,d]; o: bf16 [B,H,N,d] (written); lse: fp32 [B,H,N] (written). */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d, int causal,
+           float scale, void* stream);
+
+/* Forward, fp32 in/out: the same algorithm on the tf32 tensor-core path
+ * (operands rounded to tf32 by the tensor core, fp32 accumulation, fp32 softmax).
+ * q, k, v, o: fp32 [B,H,N,d]; lse: fp32 [B,H,N]. */
+int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int H, int N, int d,
+               int causal, float scale, void* stream);
+
+/* Bytes of device workspace fa_bwd needs for these sizes (fp32 row term D and
+ * the fp32 dQ accumulator), rounded up to 256 bytes. */
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
+
+/* Backward of fa_fwd: recomputes the scores tile by tile from q, k and the saved
+ * lse, and writes dq, dk, dv (bf16 [B,H,N,d]) for the upstream gradient dO
+ * ("flash-attention-trading-models", section "Pase hacia atras").
+ * o and lse must be the outputs of fa_fwd on the same q, k, v, causal, scale.
+ * workspace: caller-owned device buffer of at least fa_bwd_workspace_bytes()
+ * bytes, 256-byte aligned; its contents on entry do not matter. */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse, void* dq,
+           void* dk, void* dv, int B, int H, int N, int d, int causal, float scale, void* workspace,
+           size_t workspace_bytes, void* stream);
+
+/* Forward with the probability tile P cast to FP8 E4M3 before the P.V product
+ * ("P-Cast precision in FP8 attention", sections 1-2): P' = E4M3(S * p) with
+ * round-to-nearest-even and saturation at 448, accumulated against V, and the
+ * epilogue divides by S * l, where the running sum l is taken from the
+ * unquantised p.  The running max used for p includes the current tile.
+ *   S        static scale, finite and > 0 (the page recommends 256);
+ *   kv_order 0 visits key tiles 0 -> N, 1 visits them N -> 0;
+ *   stats    NULL, or a device array of 4 uint64 that the kernel ADDS to:
+ *            [0] sink P' that flushed to zero, [1] sink P counted,
+ *            [2] non-sink P' that flushed to zero, [3] non-sink P counted,
+ *            where a key is a sink when its index is < n_sink (n_sink >= 0).
+ * q, k, v, o: bf16 [B,H,N,d]; lse: fp32 [B,H,N]. */
+int fa_fwd_fp8p(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                int causal, float scale, float S, int kv_order, unsigned long long* stats, int n_sink, void* stream);
+
+/* Human-readable name of an fa_status code. */
+const char* fa_status_string(int status);
+
+/* The cudaError_t of the last FA_ERR_CUDA returned on this host thread. */
+int fa_last_cuda_error(void);
+
+/* Synchronises the current device, then reads and clears the device status word:
+ * FA_OK, or FA_ERR_TIMEOUT if a kernel's bounded wait gave up since the last
+ * call (FA_ERR_CUDA if the synchronisation itself failed). */
+int fa_check_status(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */
