@@ -16,6 +16,26 @@
 #include "fwd.cuh"
 #include "bwd.cuh"
 
+namespace fa {
+// Self-test of the failure path: waits on an mbarrier that nothing will ever
+// signal, with the given bound; the wait gives up, records FA_ERR_TIMEOUT in the
+// status word and the kernel returns normally, leaving the context usable.
+__global__ void fa_watchdog_selftest_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (!mbar_try_wait(smem_u32(&bar), 0)) mbar_wait_slow(smem_u32(&bar), 0, &abort_flag, 77, limit_ns);
+  }
+  __syncthreads();
+}
+}  // namespace fa
+
 namespace {
 
 thread_local int t_last_cuda_error = 0;
@@ -106,6 +126,62 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   return FA_OK;
 }
 
+template <int D>
+int launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse, void* dq,
+               void* dk, void* dv, int B, int H, int N, int causal, float scale, void* workspace,
+               cudaStream_t stream) {
+  using C = fa::BwdCfg<D>;
+  const int BH = B * H;
+  const int n_tiles = (N + 127) / 128;
+  const int npad = n_tiles * 128;
+  float* lse2 = static_cast<float*>(workspace);
+  float* dvec = lse2 + static_cast<size_t>(BH) * npad;
+  float* dq_acc = dvec + static_cast<size_t>(BH) * npad;
+  CUtensorMap mq, mk, mv, mdo;
+  int st;
+  const auto dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if ((st = encode_qkv_map(&mq, q, dt, 2, D, N, BH)) != FA_OK) return st;
+  if ((st = encode_qkv_map(&mk, k, dt, 2, D, N, BH)) != FA_OK) return st;
+  if ((st = encode_qkv_map(&mv, v, dt, 2, D, N, BH)) != FA_OK) return st;
+  if ((st = encode_qkv_map(&mdo, dO, dt, 2, D, N, BH)) != FA_OK) return st;
+  // 1. D, LSE*log2(e), zeroed dQ accumulator
+  const long long rows = static_cast<long long>(BH) * npad;
+  const long long pre_threads = rows * (D / 8);
+  fa::fa_bwd_pre_kernel<D><<<static_cast<unsigned>((pre_threads + 255) / 256), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2, dvec, dq_acc, N, npad,
+      rows);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  // 2. main pass over (key tile, batch*head)
+  fa::BwdArgs a;
+  a.dk = static_cast<__nv_bfloat16*>(dk);
+  a.dv = static_cast<__nv_bfloat16*>(dv);
+  a.lse2 = lse2;
+  a.dvec = dvec;
+  a.dq_acc = dq_acc;
+  a.N = N;
+  a.Npad = npad;
+  a.BH = BH;
+  a.n_tiles = n_tiles;
+  a.scale = scale;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.causal = causal ? 1 : 0;
+  auto kern = fa::fa_bwd_main_kernel<D>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return cuda_fail(e);
+  kern<<<static_cast<unsigned>(static_cast<long long>(n_tiles) * BH), C::NTHREADS, C::SMEM_BYTES, stream>>>(
+      mq, mk, mv, mdo, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  // 3. dQ accumulator -> bf16
+  const long long vecs = static_cast<long long>(BH) * N * (D / 8);
+  fa::fa_bwd_post_kernel<D><<<static_cast<unsigned>((vecs + 255) / 256), 256, 0, stream>>>(
+      dq_acc, static_cast<__nv_bfloat16*>(dq), N, npad, vecs);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return FA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -144,13 +220,33 @@ int fa_fwd_fp8p(const void* q, const void* k, const void* v, void* o, float* lse
 }
 
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
-  (void)B; (void)H; (void)N; (void)d;
-  return 0;
+  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+  const size_t npad = (static_cast<size_t>(N) + 127) / 128 * 128;
+  const size_t bytes = static_cast<size_t>(B) * H * npad * (2 + static_cast<size_t>(d)) * sizeof(float);
+  return (bytes + 255) / 256 * 256;
 }
 
-int fa_bwd(const void*, const void*, const void*, const void*, const void*, const float*, void*, void*, void*, int,
-           int, int, int, int, float, void*, size_t, void*) {
-  return FA_ERR_UNSUPPORTED;
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse, void* dq,
+           void* dk, void* dv, int B, int H, int N, int d, int causal, float scale, void* workspace,
+           size_t workspace_bytes, void* stream) {
+  int st = check_common(q, k, v, o, lse, B, H, N, d, scale);
+  if (st != FA_OK) return st;
+  if (!dO || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
+  if (!aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return FA_ERR_ALIGNMENT;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FA_ERR_ALIGNMENT;
+  if (workspace_bytes < fa_bwd_workspace_bytes(B, H, N, d)) return FA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_bwd<64>(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, causal, scale, workspace, s)
+                 : launch_bwd<128>(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, causal, scale, workspace, s);
+}
+
+int fa_watchdog_selftest(unsigned int limit_us, void* stream) {
+  if (limit_us == 0 || limit_us > 10000000u) return FA_ERR_INVALID_ARG;
+  fa::fa_watchdog_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(limit_us) * 1000ull);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return FA_OK;
 }
 
 const char* fa_status_string(int status) {

@@ -1,3 +1,434 @@
-// bwd.cuh — attention backward (placeholder until the kernels land).
+// bwd.cuh — exact attention backward on B200 by recomputation.
+//
+// The forward pass keeps only O and the row logsumexp; the backward pass
+// recomputes the score tiles from Q, K and that logsumexp instead of storing
+// the N x N probabilities ("flash-attention-trading-models", section "Pase hacia
+// atras": O(N) statistics, redundant arithmetic traded for the N^2 memory term).
+// With P = exp(scale S - LSE) and D_q = sum_c dO_qc O_qc (= sum_k P_qk dP_qk):
+//   dV = P^T dO,  dP = dO V^T,  dS = scale P o (dP - D),  dQ = dS K,  dK = dS^T Q.
+//
+// Three launches on the caller's stream:
+//   bwd_pre   D, LSE*log2(e) into padded workspace rows, zero the fp32 dQ accumulator
+//   bwd_main  one CTA per (128-key tile, batch*head): K_j, V_j stay in shared memory,
+//             the CTA walks the query tiles (from the diagonal when causal);
+//             tcgen05 MMAs: S^T = K Q^T, dP^T = V dO^T (into TMEM), then
+//             dV += P^T dO (P^T from TMEM), dK += dS^T Q, dQ_i = dS K;
+//             dV, dK accumulate in TMEM over the whole walk; each dQ_i tile is
+//             added into the fp32 accumulator in global memory.
+//   bwd_post  dQ accumulator -> bf16
+//
+// Warp roles in bwd_main (448 threads):
+//   warps 0-7   gradient warps: thread = key row (TMEM lane); warps 0-3 own query
+//               columns 0-63, warps 4-7 columns 64-127 of each tile
+//   warps 8-11  dQ drain: TMEM -> fp32 reductions into global memory
+//   warp 12     TMA producer (K_j, V_j once; Q_i, dO_i, LSE_i, D_i double-buffered)
+//   warp 13     tcgen05.mma issuer and TMEM owner
+// Tensor memory (fp32 columns): dV [0,d), dK [d,2d), S^T [2d,2d+128) with P^T
+// (bf16) written over its first 64 columns, dP^T [2d+128,2d+256); dQ_i reuses the
+// dP^T columns when d = 128 (the budget is full) and has its own when d = 64.
 #pragma once
 #include "sm100.cuh"
+
+namespace fa {
+
+// ---------------------------------------------------------------------------
+// bwd_pre: one group of D/8 threads per query row (16-byte vectors)
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
+                                                         const __nv_bfloat16* __restrict__ dO,
+                                                         const float* __restrict__ lse, float* __restrict__ lse2,
+                                                         float* __restrict__ dvec, float* __restrict__ dq_acc, int N,
+                                                         int Npad, long long rows_total) {
+  constexpr int TPR = D / 8;  // threads per row
+  const long long gtid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long row = gtid / TPR;  // padded row index over BH * Npad
+  const int part = static_cast<int>(gtid % TPR);
+  if (row >= rows_total) return;
+  const long long bh = row / Npad;
+  const int n = static_cast<int>(row % Npad);
+  float acc = 0.f;
+  if (n < N) {
+    const size_t base = (static_cast<size_t>(bh) * N + n) * D + part * 8;
+    const uint4 a = *reinterpret_cast<const uint4*>(o + base);
+    const uint4 b = *reinterpret_cast<const uint4*>(dO + base);
+    const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 x = __bfloat1622float2(pa[e]);
+      const float2 y = __bfloat1622float2(pb[e]);
+      acc = fmaf(x.x, y.x, acc);
+      acc = fmaf(x.y, y.y, acc);
+    }
+  }
+#pragma unroll
+  for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off, TPR);
+  if (part == 0) {
+    dvec[row] = acc;  // 0 on padding rows
+    lse2[row] = n < N ? lse[static_cast<size_t>(bh) * N + n] * 1.4426950408889634f : INFINITY;  // pad: P = 0
+  }
+  float4* z = reinterpret_cast<float4*>(dq_acc + static_cast<size_t>(row) * D + part * 8);
+  z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+  z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// ---------------------------------------------------------------------------
+// bwd_post: dQ accumulator (fp32, padded rows) -> bf16
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_post_kernel(const float* __restrict__ dq_acc,
+                                                          __nv_bfloat16* __restrict__ dq, int N, int Npad,
+                                                          long long vec_total) {
+  const long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;  // one 8-element vector
+  if (g >= vec_total) return;
+  constexpr int VPR = D / 8;
+  const long long row = g / VPR;  // unpadded row over BH * N
+  const int part = static_cast<int>(g % VPR);
+  const long long bh = row / N;
+  const int n = static_cast<int>(row % N);
+  const float4* src = reinterpret_cast<const float4*>(dq_acc + (static_cast<size_t>(bh) * Npad + n) * D + part * 8);
+  const float4 a = src[0], b = src[1];
+  uint4 w;
+  w.x = pack_bf16x2(a.x, a.y);
+  w.y = pack_bf16x2(a.z, a.w);
+  w.z = pack_bf16x2(b.x, b.y);
+  w.w = pack_bf16x2(b.z, b.w);
+  *reinterpret_cast<uint4*>(dq + static_cast<size_t>(row) * D + part * 8) = w;
+}
+
+// ---------------------------------------------------------------------------
+// bwd_main
+// ---------------------------------------------------------------------------
+struct BwdArgs {
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  const float* lse2;  // [BH, Npad] LSE * log2(e), +inf on padding rows
+  const float* dvec;  // [BH, Npad] D, 0 on padding rows
+  float* dq_acc;      // [BH, Npad, d]
+  int N, Npad, BH, n_tiles;
+  float scale;       // softmax scale
+  float scale_log2;  // scale * log2(e)
+  int causal;
+};
+
+template <int D>
+struct BwdCfg {
+  static constexpr int TILE = 128 * D * 2;   // one 128 x D bf16 tile
+  static constexpr int NBOX = D / 64;        // 128-byte swizzled column blocks
+  static constexpr int BOX = 16384;          // 128 rows x 128 bytes
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + TILE;
+  static constexpr int OFF_Q = OFF_V + TILE;          // 2 stages
+  static constexpr int OFF_DO = OFF_Q + 2 * TILE;     // 2 stages
+  static constexpr int OFF_DS = OFF_DO + 2 * TILE;    // dS^T, 128 keys x 128 queries bf16 (2 blocks)
+  static constexpr int OFF_LSE = OFF_DS + 2 * BOX;    // 2 stages x 128 floats
+  static constexpr int OFF_DV = OFF_LSE + 2 * 512;    // 2 stages x 128 floats
+  static constexpr int OFF_BAR = OFF_DV + 2 * 512;
+  static constexpr int SMEM_BYTES = OFF_BAR + 256;
+  static constexpr uint32_t COL_DV = 0, COL_DK = D, COL_S = 2 * D, COL_DP = 2 * D + 128;
+  static constexpr bool DQ_SHARES_DP = (2 * D + 256 + D > 512);
+  static constexpr uint32_t COL_DQ = DQ_SHARES_DP ? COL_DP : 2 * D + 256;
+  static constexpr int NTHREADS = 448;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// 16-byte chunk c (0..7) of row r inside a 128-byte-swizzled block
+__device__ __forceinline__ uint32_t sw128_off(int r, int c) {
+  return static_cast<uint32_t>(r * 128 + ((c ^ (r & 7)) << 4));
+}
+
+template <int D>
+__global__ void __launch_bounds__(448, 1)
+    fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                       const BwdArgs a) {
+  using C = BwdCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* bar_kv = bars + 0;
+  uint64_t* bar_ld_full = bars + 1;   // [2]
+  uint64_t* bar_ld_empty = bars + 3;  // [2]
+  uint64_t* bar_s_full = bars + 5;
+  uint64_t* bar_dp_full = bars + 6;
+  uint64_t* bar_pds = bars + 7;
+  uint64_t* bar_ds_free = bars + 8;
+  uint64_t* bar_dq_full = bars + 9;
+  uint64_t* bar_dq_free = bars + 10;
+  uint64_t* bar_acc = bars + 11;
+  uint64_t* bar_done = bars + 12;
+  uint32_t* tmem_base_sh = reinterpret_cast<uint32_t*>(bars + 13);
+  volatile int* abort_sh = reinterpret_cast<volatile int*>(bars + 14);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int N = a.N;
+  const int bh = blockIdx.x % a.BH;
+  const int j = blockIdx.x / a.BH;  // key tile; j = 0 (the longest walk when causal) first
+  const int i0 = a.causal ? j : 0;
+  const int steps = a.n_tiles - i0;
+
+  // the swizzled TMA/UMMA layouts need a 1024-byte aligned base
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicCAS(&g_fa_status, 0, 4 /*FA_ERR_CUDA*/ | (99 << 8));
+    return;
+  }
+  if (warp == 13) {
+    tmem_alloc(tmem_base_sh, 512);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    *abort_sh = 0;
+    mbar_init(bar_kv, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar_ld_full + s, 1);
+      mbar_init(bar_ld_empty + s, 1);
+    }
+    mbar_init(bar_s_full, 1);
+    mbar_init(bar_dp_full, 1);
+    mbar_init(bar_pds, 256);
+    mbar_init(bar_ds_free, 1);
+    mbar_init(bar_dq_full, 1);
+    mbar_init(bar_dq_free, 128);
+    mbar_init(bar_acc, 1);
+    mbar_init(bar_done, 1);
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_base_sh;
+
+  if (warp == 12) {
+    // ============================ producer ===================================
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmDO);
+      mbar_arrive_expect_tx(bar_kv, 2 * C::TILE);
+      for (int b = 0; b < C::NBOX; ++b) {
+        tma_load_3d(smem + C::OFF_K + b * C::BOX, &tmK, bar_kv, b * 64, j * 128, bh);
+        tma_load_3d(smem + C::OFF_V + b * C::BOX, &tmV, bar_kv, b * 64, j * 128, bh);
+      }
+      int t = 0;
+      for (; t < steps; ++t) {
+        const int i = i0 + t;
+        const int s = t & 1;
+        const uint32_t ph = (t >> 1) & 1;
+        if (!mbar_wait(bar_ld_empty + s, ph ^ 1, abort_sh, 40)) break;
+        mbar_arrive_expect_tx(bar_ld_full + s, 2 * C::TILE + 1024);
+        for (int b = 0; b < C::NBOX; ++b) {
+          tma_load_3d(smem + C::OFF_Q + s * C::TILE + b * C::BOX, &tmQ, bar_ld_full + s, b * 64, i * 128, bh);
+          tma_load_3d(smem + C::OFF_DO + s * C::TILE + b * C::BOX, &tmDO, bar_ld_full + s, b * 64, i * 128, bh);
+        }
+        const size_t roff = static_cast<size_t>(bh) * a.Npad + static_cast<size_t>(i) * 128;
+        bulk_load(smem + C::OFF_LSE + s * 512, a.lse2 + roff, 512, bar_ld_full + s);
+        bulk_load(smem + C::OFF_DV + s * 512, a.dvec + roff, 512, bar_ld_full + s);
+      }
+      // teardown: let the copies in flight land
+      mbar_wait_drain(bar_kv, 0, 100000000ull);
+      for (int u = max(0, t - 2); u < t; ++u) mbar_wait_drain(bar_ld_full + (u & 1), (u >> 1) & 1, 100000000ull);
+    }
+  } else if (warp == 13) {
+    // ============================ MMA issuer =================================
+    if (lane == 0) {
+      constexpr uint32_t id_ss = make_idesc(128, 128, kFmtBF16, 0, 0);      // S^T, dP^T
+      constexpr uint32_t id_dv = make_idesc(128, D, kFmtBF16, 0, 1);        // dV (A from TMEM)
+      constexpr uint32_t id_dk = make_idesc(128, D, kFmtBF16, 0, 1);        // dK
+      constexpr uint32_t id_dq = make_idesc(128, D, kFmtBF16, 1, 1);        // dQ (A = dS, MN-major)
+      const uint32_t k_addr = smem_u32(smem + C::OFF_K), v_addr = smem_u32(smem + C::OFF_V);
+      const uint32_t q_addr = smem_u32(smem + C::OFF_Q), do_addr = smem_u32(smem + C::OFF_DO);
+      const uint32_t ds_addr = smem_u32(smem + C::OFF_DS);
+      bool ok = mbar_wait(bar_kv, 0, abort_sh, 41);
+      for (int t = 0; ok && t < steps; ++t) {
+        const int s = t & 1;
+        const uint32_t ph = (t >> 1) & 1;
+        if (!(ok = mbar_wait(bar_ld_full + s, ph, abort_sh, 42))) break;
+        tc_fence_after();
+        const uint32_t qa = q_addr + s * C::TILE, da = do_addr + s * C::TILE;
+        // S^T = K_j Q_i^T    (M = 128 keys, N = 128 queries, K = d)
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * C::BOX + (k & 3) * 32;
+          mma_ss(tmem + C::COL_S, make_sdesc_sw128(k_addr + off, 16, 1024), make_sdesc_sw128(qa + off, 16, 1024),
+                 id_ss, k > 0);
+        }
+        mma_commit(bar_s_full);
+        if (C::DQ_SHARES_DP && t > 0) {
+          if (!(ok = mbar_wait(bar_dq_free, (t - 1) & 1, abort_sh, 43))) break;
+          tc_fence_after();
+        }
+        // dP^T = V_j dO_i^T
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * C::BOX + (k & 3) * 32;
+          mma_ss(tmem + C::COL_DP, make_sdesc_sw128(v_addr + off, 16, 1024), make_sdesc_sw128(da + off, 16, 1024),
+                 id_ss, k > 0);
+        }
+        mma_commit(bar_dp_full);
+        if (!(ok = mbar_wait(bar_pds, t & 1, abort_sh, 44))) break;
+        tc_fence_after();
+        // dV += P^T dO_i   (A = P^T from TMEM, K = 128 queries; B = dO_i MN-major)
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          mma_ts(tmem + C::COL_DV, tmem + C::COL_S + k * 8, make_sdesc_sw128(da + k * 2048, C::BOX, 1024), id_dv,
+                 (t > 0 || k > 0) ? 1u : 0u);
+        // dK += dS^T Q_i   (A = dS^T K-major in smem; B = Q_i MN-major)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t off = (k >> 2) * C::BOX + (k & 3) * 32;
+          mma_ss(tmem + C::COL_DK, make_sdesc_sw128(ds_addr + off, 16, 1024),
+                 make_sdesc_sw128(qa + k * 2048, C::BOX, 1024), id_dk, (t > 0 || k > 0) ? 1u : 0u);
+        }
+        if (!C::DQ_SHARES_DP && t > 0) {
+          if (!(ok = mbar_wait(bar_dq_free, (t - 1) & 1, abort_sh, 45))) break;
+          tc_fence_after();
+        }
+        // dQ_i = dS K_j     (A = dS: the dS^T buffer read MN-major; B = K_j MN-major)
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          mma_ss(tmem + C::COL_DQ, make_sdesc_sw128(ds_addr + k * 2048, C::BOX, 1024),
+                 make_sdesc_sw128(k_addr + k * 2048, C::BOX, 1024), id_dq, k > 0 ? 1u : 0u);
+        mma_commit(bar_dq_full);
+        mma_commit(bar_ld_empty + s);
+        mma_commit(bar_ds_free);
+      }
+      if (ok) mma_commit(bar_acc);
+      mma_commit(bar_done);
+      mbar_wait_drain(bar_done, 0, 100000000ull);
+    }
+  } else if (warp >= 8) {
+    // ============================ dQ drain ===================================
+    const int r = threadIdx.x - 256;  // query row in tile == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    for (int t = 0; t < steps; ++t) {
+      const int i = i0 + t;
+      if (!mbar_wait(bar_dq_full, t & 1, abort_sh, 46)) break;
+      tc_fence_after();
+      float* dst = a.dq_acc + (static_cast<size_t>(bh) * a.Npad + static_cast<size_t>(i) * 128 + r) * D;
+      const bool live = i * 128 + r < N;
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_base + C::COL_DQ + ch * 32, v);
+        tmem_wait_ld();
+        if (live) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            atomicAdd(reinterpret_cast<float4*>(dst + ch * 32 + 4 * e),
+                      make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                                  __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3])));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_dq_free);
+    }
+  } else {
+    // ============================ gradient warps =============================
+    const int half = warp >> 2;                  // query columns [64 half, 64 half + 64)
+    const int r = threadIdx.x & 127;             // key row in tile == TMEM lane
+    const int key = j * 128 + r;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    const float c = a.scale_log2;
+    bool ok = true;
+    for (int t = 0; t < steps && ok; ++t) {
+      const int i = i0 + t;
+      const int s = t & 1;
+      const float* lse2 = reinterpret_cast<const float*>(smem + C::OFF_LSE + s * 512) + half * 64;
+      const float* dv = reinterpret_cast<const float*>(smem + C::OFF_DV + s * 512) + half * 64;
+      const int q0 = i * 128 + half * 64;
+      const bool need_mask = (a.causal && i == j) || key >= N;
+      if (!(ok = mbar_wait(bar_s_full, t & 1, abort_sh, 47))) break;
+      tc_fence_after();
+      float p[64];
+      tmem_ld32(tmem + lane_base + C::COL_S + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&p[0]));
+      tmem_ld32(tmem + lane_base + C::COL_S + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&p[32]));
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 64; ++e) {
+        float x = ex2_approx(fmaf(p[e], c, -lse2[e]));
+        if (need_mask && (key >= N || (a.causal && key > q0 + e))) x = 0.f;
+        p[e] = x;
+      }
+      // both halves have read S^T before P^T is written over its first 64 columns
+      named_bar_sync(1, 256);
+      {
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
+        tmem_st32(tmem + lane_base + C::COL_S + half * 32, pk);
+      }
+      if (!(ok = mbar_wait(bar_ds_free, (t & 1) ^ 1, abort_sh, 48))) break;
+      if (!(ok = mbar_wait(bar_dp_full, t & 1, abort_sh, 49))) break;
+      tc_fence_after();
+      uint8_t* dsb = smem + C::OFF_DS + half * C::BOX;  // queries [64 half, +64) live in block `half`
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t dp[32];
+        tmem_ld32(tmem + lane_base + C::COL_DP + half * 64 + h2 * 32, dp);
+        tmem_wait_ld();
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {  // 4 chunks of 8 queries
+          uint4 w;
+          uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int qi = h2 * 32 + cc * 8 + 2 * e;
+            const float d0 = a.scale * p[qi] * (__uint_as_float(dp[cc * 8 + 2 * e]) - dv[qi]);
+            const float d1 = a.scale * p[qi + 1] * (__uint_as_float(dp[cc * 8 + 2 * e + 1]) - dv[qi + 1]);
+            wp[e] = pack_bf16x2(d0, d1);
+          }
+          *reinterpret_cast<uint4*>(dsb + sw128_off(r, h2 * 4 + cc)) = w;
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      fence_proxy_async_smem();
+      mbar_arrive(bar_pds);
+    }
+    // ---- epilogue: dV (warps 0-3) and dK (warps 4-7) -> bf16 -------------------
+    if (ok) ok = mbar_wait(bar_acc, 0, abort_sh, 50);
+    if (ok) {
+      tc_fence_after();
+      const uint32_t col = half ? C::COL_DK : C::COL_DV;
+      __nv_bfloat16* dst = (half ? a.dk : a.dv) + (static_cast<size_t>(bh) * N + key) * D;
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_base + col + ch * 32, v);
+        tmem_wait_ld();
+        if (key < N) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + ch * 32);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(v[8 * v4 + 0]), __uint_as_float(v[8 * v4 + 1]));
+            w.y = pack_bf16x2(__uint_as_float(v[8 * v4 + 2]), __uint_as_float(v[8 * v4 + 3]));
+            w.z = pack_bf16x2(__uint_as_float(v[8 * v4 + 4]), __uint_as_float(v[8 * v4 + 5]));
+            w.w = pack_bf16x2(__uint_as_float(v[8 * v4 + 6]), __uint_as_float(v[8 * v4 + 7]));
+            d4[v4] = w;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 13) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fa

@@ -71,13 +71,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Bounded wait for the phase with the given parity to complete.  `abort_flag`
 // is a CTA-shared word; once any thread of the CTA gave up, the others stop
 // waiting too.  Returns false on timeout/abort.
-__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag, int site) {
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag, int site,
+                                            uint64_t limit_ns = FA_WAIT_LIMIT_NS) {
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > FA_WAIT_LIMIT_NS) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         atomicCAS(&g_fa_status, 0, 5 /*FA_ERR_TIMEOUT*/ | (site << 8));
         *abort_flag = 1;
         return false;

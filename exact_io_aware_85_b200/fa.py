@@ -28,10 +28,11 @@ lib.fa_status_string.restype = ctypes.c_char_p
 lib.fa_status_string.argtypes = [_ci]
 lib.fa_last_cuda_error.restype = _ci
 lib.fa_check_status.restype = _ci
+lib.fa_watchdog_selftest.argtypes = [ctypes.c_uint, _vp]
 
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_ALIGNMENT, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(6)
 EXPORTS = ("fa_fwd", "fa_fwd_f32", "fa_fwd_fp8p", "fa_bwd_workspace_bytes", "fa_bwd", "fa_status_string",
-           "fa_last_cuda_error", "fa_check_status")
+           "fa_last_cuda_error", "fa_check_status", "fa_watchdog_selftest")
 
 
 class FAError(RuntimeError):
@@ -104,3 +105,7 @@ def fa_status_string(status: int) -> str:
 
 def fa_check_status() -> int:
     return int(lib.fa_check_status())
+
+
+def fa_watchdog_selftest(limit_us: int, stream=None) -> None:
+    _check(lib.fa_watchdog_selftest(int(limit_us), _stream(stream)), "fa_watchdog_selftest")

@@ -99,6 +99,13 @@ int fa_last_cuda_error(void);
  * call (FA_ERR_CUDA if the synchronisation itself failed). */
 int fa_check_status(void);
 
+/* Failure-path self-test: launches a one-block kernel whose bounded wait on a
+ * barrier that nothing signals gives up after limit_us microseconds (1 .. 10^7),
+ * records FA_ERR_TIMEOUT in the device status word and returns; the CUDA context
+ * stays usable.  fa_check_status() then reports FA_ERR_TIMEOUT.  Every wait in
+ * the attention kernels is bounded the same way (at 2 s). */
+int fa_watchdog_selftest(unsigned int limit_us, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
