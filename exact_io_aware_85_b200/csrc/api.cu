@@ -182,6 +182,37 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   return FA_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free backward: the workspace lives in a fixed device array that
+// the library defines itself.  Host code must not hand the array's name to a
+// kernel (on the host it only stands for the symbol); each device's address of
+// it is looked up once with cudaGetSymbolAddress and cached.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB, held by every GPU that loads the library
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_bwd_scratch[kNoAllocScratchBytes];
+
+namespace {
+int noalloc_scratch_for_current_device(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_bwd_scratch);
+    if (e != cudaSuccess) return cuda_fail(e);
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return FA_OK;
+}
 }  // namespace
 
 extern "C" {
@@ -238,6 +269,20 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return d == 64 ? launch_bwd<64>(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, causal, scale, workspace, s)
                  : launch_bwd<128>(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, causal, scale, workspace, s);
+}
+
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                   void* dq, void* dk, void* dv, int B, int H, int N, int d, int causal, float scale, void* stream) {
+  int st = check_common(q, k, v, o, lse, B, H, N, d, scale);
+  if (st != FA_OK) return st;
+  if (!dO || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (!aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return FA_ERR_ALIGNMENT;
+  if (fa_bwd_workspace_bytes(B, H, N, d) > kNoAllocScratchBytes) return FA_ERR_UNSUPPORTED;
+  void* ws = nullptr;
+  if ((st = noalloc_scratch_for_current_device(&ws)) != FA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_bwd<64>(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, causal, scale, ws, s)
+                 : launch_bwd<128>(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, causal, scale, ws, s);
 }
 
 int fa_watchdog_selftest(unsigned int limit_us, void* stream) {

@@ -109,3 +109,15 @@ def fa_check_status() -> int:
 
 def fa_watchdog_selftest(limit_us: int, stream=None) -> None:
     _check(lib.fa_watchdog_selftest(int(limit_us), _stream(stream)), "fa_watchdog_selftest")
+
+
+lib.fa_bwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _cf, _vp]
+
+
+def fa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, causal: bool, scale: float, stream=None) -> None:
+    """Backward without a caller workspace: the library's own fixed device scratch
+    array (32 MiB) is used, so nothing is allocated; larger sizes raise
+    FA_ERR_UNSUPPORTED.  Calls that overlap on the GPU race on that array."""
+    B, H, N, d = _dims(q)
+    _check(lib.fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+                              B, H, N, d, int(causal), float(scale), _stream(stream)), "fa_bwd_noalloc")

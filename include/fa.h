@@ -73,6 +73,30 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
            void* dk, void* dv, int B, int H, int N, int d, int causal, float scale, void* workspace,
            size_t workspace_bytes, void* stream);
 
+/* Backward for callers that cannot allocate device memory: some embedders run
+ * under an allocator they do not own (a framework's caching pool, a process
+ * whose memory budget is fixed up front) or in code paths where a cudaMalloc
+ * would synchronise the device or is forbidden outright, so they cannot supply
+ * fa_bwd's workspace.  This variant takes the same arguments as fa_bwd minus the
+ * workspace and uses a scratch array that the library itself defines in device
+ * memory: FA_BWD_NOALLOC_MAX_BYTES (32 MiB), reserved on every GPU that loads the
+ * library for as long as it stays loaded.  It calls no allocation routine.
+ *  - Sizes whose workspace (fa_bwd_workspace_bytes) exceeds that maximum are
+ *    rejected with FA_ERR_UNSUPPORTED before anything is launched.
+ *  - The first call on a device looks up that device's address of the array
+ *    (cudaGetSymbolAddress) and caches it; make that first call before any
+ *    stream capture.
+ *  - All calls on a device share the one array and it keeps the previous call's
+ *    contents; each call rewrites every part it reads (the first of its kernels
+ *    rewrites the row statistics and zeroes the dQ accumulator).  Calls whose
+ *    work overlaps on the GPU (different streams, or different host threads)
+ *    race on the array: serialise them.
+ * The pages have no counterpart to this entry point; results are those of
+ * fa_bwd on the same inputs. */
+#define FA_BWD_NOALLOC_MAX_BYTES (32u << 20)
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                   void* dq, void* dk, void* dv, int B, int H, int N, int d, int causal, float scale, void* stream);
+
 /* Forward with the probability tile P cast to FP8 E4M3 before the P.V product
  * ("P-Cast precision in FP8 attention", sections 1-2): P' = E4M3(S * p) with
  * round-to-nearest-even and saturation at 448, accumulated against V, and the

@@ -1,0 +1,64 @@
+"""fa_bwd_noalloc: the backward for callers that cannot allocate device memory
+(it runs on a fixed scratch array inside the library instead of a workspace the
+caller passes).  Checked through the C ABI against fa_bwd on two calls in a
+row with different sizes, so that what the first call leaves in the shared
+scratch array cannot leak into the second; and a size whose workspace exceeds
+the array is refused before any launch.  This file is collected last on purpose."""
+import ctypes
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from exact_io_aware_85_b200 import synth
+
+pytestmark = pytest.mark.gpu
+REL_L2 = 2e-2  # the backward tolerance used by the parity tests
+
+
+def _rel_l2(a, b):
+    a, b = a.double(), b.double()
+    return float((a - b).norm() / max(float(b.norm()), 1e-30))
+
+
+def _case(B, H, N, d, causal, seed):
+    from exact_io_aware_85_b200 import fa
+    x = synth.make_inputs(B, H, N, d, "bf16", seed=seed, with_grad=True)
+    q, k, v, do = (torch.from_numpy(x[n]).to(torch.bfloat16).cuda() for n in ("q", "k", "v", "do"))
+    scale = 1.0 / math.sqrt(d)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    fa.fa_fwd(q, k, v, o, lse, causal, scale)
+    # existing entry point, caller-owned workspace
+    ref = [torch.empty_like(q) for _ in range(3)]
+    ws = torch.empty(fa.fa_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device="cuda")
+    fa.fa_bwd(q, k, v, o, do, lse, *ref, causal, scale, ws)
+    # allocation-free entry point, called through the raw C ABI
+    got = [torch.full_like(q, float("nan")) for _ in range(3)]
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    st = fa.lib.fa_bwd_noalloc(p(q), p(k), p(v), p(o), p(do), p(lse), *(p(t) for t in got), B, H, N, d, int(causal),
+                               ctypes.c_float(scale), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == fa.FA_OK, fa.fa_status_string(st)
+    torch.cuda.synchronize()
+    assert fa.fa_check_status() == fa.FA_OK
+    for name, g, r in zip(("dq", "dk", "dv"), got, ref):
+        assert torch.isfinite(g.float()).all(), name
+        assert _rel_l2(g.float(), r.float()) <= REL_L2, name
+    # dK and dV come from the same kernels in the same order: identical bits
+    assert torch.equal(got[1], ref[1]) and torch.equal(got[2], ref[2])
+
+
+def test_noalloc_matches_fa_bwd_on_two_calls_in_a_row():
+    _case(1, 2, 700, 128, True, seed=901)   # first call on this device sets up the scratch address
+    _case(2, 1, 257, 64, False, seed=902)   # second call reuses the array left by the first
+
+
+def test_noalloc_refuses_sizes_beyond_the_scratch_array():
+    from exact_io_aware_85_b200 import fa
+    B, H, N, d = 2, 16, 4096, 128  # needs 68 MB of workspace > 32 MiB
+    assert fa.fa_bwd_workspace_bytes(B, H, N, d) > 32 << 20
+    dummy = torch.empty(16, dtype=torch.bfloat16, device="cuda")
+    p = ctypes.c_void_p(dummy.data_ptr())
+    st = fa.lib.fa_bwd_noalloc(p, p, p, p, p, p, p, p, p, B, H, N, d, 1, ctypes.c_float(0.088), None)
+    assert st == fa.FA_ERR_UNSUPPORTED
