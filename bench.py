@@ -161,16 +161,15 @@ def cpu_baseline(w: synth.Workload, target_s: float = 12.0):
         nk = (rows[:, 1] + 1) if w.causal else np.full(len(rows), w.N)
         return float((4.0 * w.d * nk).sum())
 
-    rows = np.stack([np.zeros(64, dtype=np.int64), rng.integers(0, w.N, 64)], axis=1)
-    t0 = time.perf_counter()
-    oracle.attn_fwd_rows(x["q"], x["k"], x["v"], rows, w.causal, w.scale)
-    dt = time.perf_counter() - t0
-    rate = flops(rows) / max(dt, 1e-6)
-    n = int(min(200000, max(64, 64 * target_s / max(dt, 1e-6))))
-    rows = np.stack([np.zeros(n, dtype=np.int64), rng.integers(0, w.N, n)], axis=1)
-    t0 = time.perf_counter()
-    oracle.attn_fwd_rows(x["q"], x["k"], x["v"], rows, w.causal, w.scale)
-    dt = time.perf_counter() - t0
+    n, dt = 256, 0.0
+    while True:  # grow the sample until it takes about target_s of host time
+        rows = np.stack([np.zeros(n, dtype=np.int64), rng.integers(0, w.N, n)], axis=1)
+        t0 = time.perf_counter()
+        oracle.attn_fwd_rows(x["q"], x["k"], x["v"], rows, w.causal, w.scale)
+        dt = time.perf_counter() - t0
+        if dt >= 0.5 * target_s or n >= 400000:
+            break
+        n = int(min(400000, n * max(2.0, 0.9 * target_s / max(dt, 1e-3))))
     rate = flops(rows) / dt
     return {"value": rate / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
             "sample": f"{n} random query rows of one head of the {w.name} workload (N={w.N}, d={w.d}, "
@@ -208,8 +207,10 @@ METRIC = "attention fwd/bwd TFLOP/s at 1 B200 and % of dense BF16/FP8 tensor pea
 
 
 def config_of(w, ws):
+    what = ("forward + backward (dQ, dK, dV from the saved LSE)" if w.backward else
+            "FP8 P-cast forward, S=256, forward key order, sink Delta=8" if w.sink else "forward (O + LSE)")
     return {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} {w.dtype} "
-                        f"{'causal' if w.causal else 'non-causal'} forward (O + LSE)",
+                        f"{'causal' if w.causal else 'non-causal'} {what}",
             "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal, "parallelism": f"replicas x{ws}",
             "l2": "inputs larger than L2 (no flush needed)" if 3 * w.B * w.H * w.N * w.d * 2 > 126e6
             else "L2 flushed between steps"}
@@ -237,8 +238,34 @@ def main():
     o = torch.empty_like(q)
     lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
-    run = (lambda: fa.fa_fwd(q, k, v, o, lse, w.causal, w.scale)) if w.dtype == "bf16" else \
-        (lambda: fa.fa_fwd_f32(q, k, v, o, lse, w.causal, w.scale))
+    launches_per_step = 1
+    if w.backward:
+        # training step: forward, then backward from the saved LSE (4 launches)
+        g = torch.Generator(device="cuda")
+        g.manual_seed(synth.workload_seed(w.name) + 7919 + rank)
+        do = torch.randn(q.shape, generator=g, device="cuda", dtype=torch.float32).to(q.dtype)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+        ws_buf = torch.empty(fa.fa_bwd_workspace_bytes(w.B, w.H, w.N, w.d), dtype=torch.uint8, device="cuda")
+        launches_per_step = 4
+
+        def run():
+            fa.fa_fwd(q, k, v, o, lse, w.causal, w.scale)
+            fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, w.causal, w.scale, ws_buf)
+    elif w.sink:
+        # FP8 P-cast, forward key order, S = 256, on sink inputs with Delta = 8
+        k[..., :4, 0] = 8.0 * math.sqrt(w.d)
+        k[..., 4:, 0] = 0.0
+        q[..., 0] = 1.0
+        stats = torch.zeros(4, dtype=torch.int64, device="cuda")
+
+        def run():
+            fa.fa_fwd_fp8p(q, k, v, o, lse, w.causal, w.scale, 256.0, 0, stats, 4)
+    elif w.dtype == "bf16":
+        def run():
+            fa.fa_fwd(q, k, v, o, lse, w.causal, w.scale)
+    else:
+        def run():
+            fa.fa_fwd_f32(q, k, v, o, lse, w.causal, w.scale)
     small = 3 * q.numel() * q.element_size() < 126e6
     flush = torch.empty(int(256e6), dtype=torch.uint8, device="cuda") if small else None
 
@@ -269,7 +296,7 @@ def main():
     step_ms_local = sum(launch_ms) / len(launch_ms)
     step_ms = max_over_ranks(step_ms_local, ws)
     assert fa.fa_check_status() == 0
-    flops = w.fwd_flops()
+    flops = w.fwd_flops() + (w.bwd_flops() if w.backward else 0.0)
     value = ws * flops / (step_ms * 1e-3) / 1e12
 
     # ---- end to end through the C ABI with pinned host buffers -----------------
@@ -278,12 +305,23 @@ def main():
     hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
     e2e_steps = max(3, min(args.steps, 10))
 
+    if w.backward:
+        hdo = do.cpu().pin_memory()
+        hdq, hdk, hdv = (torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for _ in range(3))
+
     def e2e_step():
         q.copy_(hq, non_blocking=True)
         k.copy_(hk, non_blocking=True)
         v.copy_(hv, non_blocking=True)
+        if w.backward:
+            do.copy_(hdo, non_blocking=True)
         run()
-        ho.copy_(o, non_blocking=True)
+        if w.backward:
+            hdq.copy_(dq, non_blocking=True)
+            hdk.copy_(dk, non_blocking=True)
+            hdv.copy_(dv, non_blocking=True)
+        else:
+            ho.copy_(o, non_blocking=True)
         hl.copy_(lse, non_blocking=True)
 
     e2e_step()
@@ -298,9 +336,17 @@ def main():
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, ws)
     h2d = 3 * q.numel() * q.element_size()
-    d2h = o.numel() * o.element_size() + lse.numel() * 4
+    d2h = (3 * q.numel() * q.element_size() if w.backward else o.numel() * o.element_size()) + lse.numel() * 4
+    if w.backward:
+        h2d += do.numel() * do.element_size()
 
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    if w.backward:
+        kernel_name = "training step: fa_fwd_kernel<bf16,%d> + fa_bwd (pre, main, post)" % w.d
+    elif w.sink:
+        kernel_name = "fa_fwd_kernel<bf16,%d,FP8P>" % w.d
+    else:
+        kernel_name = "fa_fwd_kernel<%s,%d>" % ("bf16" if w.dtype == "bf16" else "f32/tf32", w.d)
     achieved = flops / (step_ms_local * 1e-3) / 1e12
     tr = TRAFFIC.get(w.name, {})
     traffic = tr.get("bytes") if tr.get("fwd_src_sha1") == _src_hash() else None
@@ -319,13 +365,13 @@ def main():
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)"
                          if peak_src == "measured" else "fallback 1590 TFLOP/s",
-                         "traffic": traffic, "kernel": "fa_fwd_kernel<bf16,%d>" % w.d,
+                         "traffic": traffic, "kernel": kernel_name,
                          "launch_ms": {"median": statistics.median(launch_ms), "min": min(launch_ms),
                                        "mean": step_ms_local}},
             "clocks": clocks,
             "e2e": {"value": ws * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": args.steps,
+            "gpu_launches": args.steps * launches_per_step,
         }
         if ws == 1 and not args.no_cpu_baseline:
             cb = cpu_baseline(w)

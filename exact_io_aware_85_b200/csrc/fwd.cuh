@@ -99,8 +99,15 @@ __global__ void __launch_bounds__(320, 1)
 
   // ---- work decode: heaviest query blocks first when causal -----------------
   const int N = a.N;
-  const int bh = blockIdx.x % a.BH;
-  int qblk = blockIdx.x / a.BH;
+  // CTAs in flight should share K/V through L2: blocks are issued in groups of
+  // kHeadGroup heads (all query blocks of the group, heaviest first when causal),
+  // so the resident working set is a few heads' K/V instead of one per SM.
+  constexpr int kHeadGroup = 8;
+  const int group = blockIdx.x / (kHeadGroup * a.nblk);
+  const int heads_in_group = min(kHeadGroup, a.BH - group * kHeadGroup);
+  const int r_in_group = blockIdx.x - group * kHeadGroup * a.nblk;
+  const int bh = group * kHeadGroup + r_in_group % heads_in_group;
+  int qblk = r_in_group / heads_in_group;
   if (a.causal) qblk = a.nblk - 1 - qblk;
   const int m0 = qblk * 256;
   const int n_kv = (N + 127) >> 7;
@@ -342,29 +349,26 @@ __global__ void __launch_bounds__(320, 1)
           for (int cc = 0; cc < 128; ++cc)
             if (kbase + cc > lim) sv[cc] = -INFINITY;
         }
-        float mx = sv[0];
+        // row max as 8 independent chains (a single 128-long chain is pure latency)
+        float mx8[8];
 #pragma unroll
-        for (int cc = 1; cc < 128; ++cc) mx = fmaxf(mx, sv[cc]);
+        for (int u = 0; u < 8; ++u) mx8[u] = fmaxf(sv[u], sv[u + 8]);
+#pragma unroll
+        for (int cc = 16; cc < 128; cc += 8)
+#pragma unroll
+          for (int u = 0; u < 8; ++u) mx8[u] = fmaxf(mx8[u], sv[cc + u]);
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         float m_new = fmaxf(m_run, mx * c);
         // Lazy rescale: keep the old max while the growth stays within 2^8 (exps stay
         // <= 256, safe in bf16/fp32).  The FP8 P-cast needs the exact running max.
         if (!FP8P && m_new - m_run <= 8.0f) m_new = m_run;
         const float alpha = ex2_approx(m_run - m_new);
-        if (cnt > 0 && __any_sync(0xffffffffu, m_new != m_run)) {
-#pragma unroll
-          for (int ch = 0; ch < D / 32; ++ch) {
-            uint32_t ov[32];
-            tmem_ld32(tO + ch * 32, ov);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-            tmem_st32(tO + ch * 32, ov);
-          }
-        }
+        const bool rescale = cnt > 0 && __any_sync(0xffffffffu, m_new != m_run);
         l_run *= alpha;
         m_run = m_new;
         const float neg_m = -m_run;
-        float rs = 0.f;
+        float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 8 independent partial row sums
         if constexpr (C::EB == 2) {
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
@@ -373,7 +377,7 @@ __global__ void __launch_bounds__(320, 1)
             for (int e = 0; e < 32; ++e) {
               const float p0 = ex2_approx(fmaf(sv[h * 64 + 2 * e], c, neg_m));
               const float p1 = ex2_approx(fmaf(sv[h * 64 + 2 * e + 1], c, neg_m));
-              rs += p0 + p1;
+              rs8[e & 7] += p0 + p1;
               if constexpr (FP8P) {
                 float q0, q1;
                 pk[e] = e4m3_roundtrip_bf16x2(p0 * a.p_scale, p1 * a.p_scale, q0, q1);
@@ -396,16 +400,29 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               const float p = ex2_approx(fmaf(sv[h * 32 + e], c, neg_m));
-              rs += p;
+              rs8[e & 7] += p;
               pk[e] = __float_as_uint(p);
             }
             tmem_st32(tS + h * 32, pk);
           }
         }
+        // O correction after P is out (the S values are dead by now, which keeps
+        // register pressure down); PV_i(j-1) is complete since S_i(j) arrived.
+        if (rescale) {
+#pragma unroll
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t ov[32];
+            tmem_ld32(tO + ch * 32, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            tmem_st32(tO + ch * 32, ov);
+          }
+        }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bar_p[i]);
-        l_run += rs;
+        l_run += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
         ++cnt;
       }
       // ---- epilogue: O / l -> global, LSE -> global --------------------------
