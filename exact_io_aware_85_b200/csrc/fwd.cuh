@@ -337,28 +337,43 @@ __global__ void __launch_bounds__(320, 1)
         if (!(ok = mbar_wait(&bar_s[i], cnt & 1, &abort_sh, 10 + i))) break;
         tc_fence_after();
         float sv[128];
+        // first half of the row, then the second half streams in while the
+        // first half's max is formed
         tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
         tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_wait_ld();
         tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
         tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
-        tmem_wait_ld();
         const int kbase = j * 128;
-        if (kbase + 128 > N || (a.causal && j == qt)) {
-          const int lim = a.causal ? min(N - 1, row) : N - 1;  // last admissible key
+        const bool masked_tile = kbase + 128 > N || (a.causal && j == qt);
+        const int lim = a.causal ? min(N - 1, row) : N - 1;  // last admissible key
+        if (masked_tile) {
 #pragma unroll
-          for (int cc = 0; cc < 128; ++cc)
+          for (int cc = 0; cc < 64; ++cc)
             if (kbase + cc > lim) sv[cc] = -INFINITY;
         }
-        // row max as 8 independent chains (a single 128-long chain is pure latency)
+        // row max as 8 independent chains of 3-input max (a single 128-long chain
+        // would be pure latency)
         float mx8[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) mx8[u] = fmaxf(sv[u], sv[u + 8]);
+        for (int u = 0; u < 8; ++u) mx8[u] = fmax3(sv[u], sv[u + 8], sv[u + 16]);
 #pragma unroll
-        for (int cc = 16; cc < 128; cc += 8)
+        for (int cc = 24; cc < 56; cc += 16)
 #pragma unroll
-          for (int u = 0; u < 8; ++u) mx8[u] = fmaxf(mx8[u], sv[cc + u]);
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+          for (int u = 0; u < 8; ++u) mx8[u] = fmax3(mx8[u], sv[cc + u], sv[cc + 8 + u]);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mx8[u] = fmaxf(mx8[u], sv[56 + u]);
+        tmem_wait_ld();
+        if (masked_tile) {
+#pragma unroll
+          for (int cc = 64; cc < 128; ++cc)
+            if (kbase + cc > lim) sv[cc] = -INFINITY;
+        }
+#pragma unroll
+        for (int cc = 64; cc < 128; cc += 16)
+#pragma unroll
+          for (int u = 0; u < 8; ++u) mx8[u] = fmax3(mx8[u], sv[cc + u], sv[cc + 8 + u]);
+        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
         float m_new = fmaxf(m_run, mx * c);
         // Lazy rescale: keep the old max while the growth stays within 2^8 (exps stay
         // <= 256, safe in bf16/fp32).  The FP8 P-cast needs the exact running max.
@@ -368,22 +383,24 @@ __global__ void __launch_bounds__(320, 1)
         l_run *= alpha;
         m_run = m_new;
         const float neg_m = -m_run;
-        float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 8 independent partial row sums
+        // 4 independent pairs of partial row sums (packed fp32x2 adds)
+        float2 rs4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        const float2 c2 = make_float2(c, c), nm2 = make_float2(neg_m, neg_m);
         if constexpr (C::EB == 2) {
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             uint32_t pk[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              const float p0 = ex2_approx(fmaf(sv[h * 64 + 2 * e], c, neg_m));
-              const float p1 = ex2_approx(fmaf(sv[h * 64 + 2 * e + 1], c, neg_m));
-              rs8[e & 7] += p0 + p1;
+              const float2 x = ffma2(make_float2(sv[h * 64 + 2 * e], sv[h * 64 + 2 * e + 1]), c2, nm2);
+              const float p0 = ex2_approx(x.x);
+              const float p1 = ex2_approx(x.y);
+              rs4[e & 3] = fadd2(rs4[e & 3], make_float2(p0, p1));
               if constexpr (FP8P) {
                 float q0, q1;
                 pk[e] = e4m3_roundtrip_bf16x2(p0 * a.p_scale, p1 * a.p_scale, q0, q1);
                 if (a.stats != nullptr && row < N) {
                   const int k0 = kbase + h * 64 + 2 * e;
-                  const int lim = a.causal ? min(N - 1, row) : N - 1;
                   if (k0 <= lim && q0 == 0.f) { if (k0 < a.n_sink) ++fl_sink; else ++fl_non; }
                   if (k0 + 1 <= lim && q1 == 0.f) { if (k0 + 1 < a.n_sink) ++fl_sink; else ++fl_non; }
                 }
@@ -400,7 +417,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               const float p = ex2_approx(fmaf(sv[h * 32 + e], c, neg_m));
-              rs8[e & 7] += p;
+              rs4[e & 3].x += p;
               pk[e] = __float_as_uint(p);
             }
             tmem_st32(tS + h * 32, pk);
@@ -415,14 +432,23 @@ __global__ void __launch_bounds__(320, 1)
             tmem_ld32(tO + ch * 32, ov);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            for (int e = 0; e < 32; e += 2) {
+              const float2 r2 = fmul2(make_float2(__uint_as_float(ov[e]), __uint_as_float(ov[e + 1])),
+                                      make_float2(alpha, alpha));
+              ov[e] = __float_as_uint(r2.x);
+              ov[e + 1] = __float_as_uint(r2.y);
+            }
             tmem_st32(tO + ch * 32, ov);
           }
         }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bar_p[i]);
-        l_run += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+        {
+          const float2 t01 = fadd2(rs4[0], rs4[1]), t23 = fadd2(rs4[2], rs4[3]);
+          const float2 t = fadd2(t01, t23);
+          l_run += t.x + t.y;
+        }
         ++cnt;
       }
       // ---- epilogue: O / l -> global, LSE -> global --------------------------
