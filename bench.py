@@ -123,12 +123,20 @@ def dist_setup():
 
 
 def max_over_ranks(x: float, ws: int) -> float:
+    """Max of a per-rank scalar (the device step time) over all ranks."""
     if ws == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(flops_per_rank: float, step_ms_max: float, ws: int) -> float:
+    """Whole-job TFLOP/s under weak scaling: every rank does flops_per_rank per
+    step and the job's step takes the slowest rank's time."""
+    return ws * flops_per_rank / (step_ms_max * 1e-3) / 1e12
 
 
 def barrier(ws: int):
@@ -297,7 +305,7 @@ def main():
     step_ms = max_over_ranks(step_ms_local, ws)
     assert fa.fa_check_status() == 0
     flops = w.fwd_flops() + (w.bwd_flops() if w.backward else 0.0)
-    value = ws * flops / (step_ms * 1e-3) / 1e12
+    value = job_throughput(flops, step_ms, ws)
 
     # ---- end to end through the C ABI with pinned host buffers -----------------
     hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
@@ -369,7 +377,7 @@ def main():
                          "launch_ms": {"median": statistics.median(launch_ms), "min": min(launch_ms),
                                        "mean": step_ms_local}},
             "clocks": clocks,
-            "e2e": {"value": ws * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+            "e2e": {"value": job_throughput(flops, e2e_ms, ws), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": args.steps * launches_per_step,
         }
