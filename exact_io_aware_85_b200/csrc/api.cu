@@ -63,13 +63,13 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // [B*H, N, d] row-major tensor seen as a 3-D TMA tensor (d, N, B*H); box of
 // 128 bytes x 128 rows with the 128-byte swizzle.  Rows beyond N read as zero.
 int encode_qkv_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, int d, int N, int BH,
-                   CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
+                   CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B, int box_rows = 128) {
   auto fn = encode_fn();
   if (!fn) return cuda_fail(cudaErrorNotSupported);
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * elem_bytes,
                            static_cast<cuuint64_t>(d) * static_cast<cuuint64_t>(N) * elem_bytes};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem_bytes), 128, 1};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem_bytes), static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -166,11 +166,24 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.causal = causal ? 1 : 0;
-  auto kern = fa::fa_bwd_main_kernel<D>;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-  if (e != cudaSuccess) return cuda_fail(e);
-  kern<<<static_cast<unsigned>(static_cast<long long>(n_tiles) * BH), C::NTHREADS, C::SMEM_BYTES, stream>>>(
-      mq, mk, mv, mdo, a);
+  if constexpr (D == 128) {
+    // pipelined 64-query variant: Q and dO tiles of 64 rows
+    CUtensorMap mq64, mdo64;
+    if ((st = encode_qkv_map(&mq64, q, dt, 2, D, N, BH, CU_TENSOR_MAP_SWIZZLE_128B, 64)) != FA_OK) return st;
+    if ((st = encode_qkv_map(&mdo64, dO, dt, 2, D, N, BH, CU_TENSOR_MAP_SWIZZLE_128B, 64)) != FA_OK) return st;
+    using CQ = fa::BwdQ64Cfg;
+    auto kern = fa::fa_bwd_main_q64_kernel;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, CQ::SMEM_BYTES);
+    if (e != cudaSuccess) return cuda_fail(e);
+    kern<<<static_cast<unsigned>(static_cast<long long>(n_tiles) * BH), CQ::NTHREADS, CQ::SMEM_BYTES, stream>>>(
+        mq64, mk, mv, mdo64, a);
+  } else {
+    auto kern = fa::fa_bwd_main_kernel<D>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return cuda_fail(e);
+    kern<<<static_cast<unsigned>(static_cast<long long>(n_tiles) * BH), C::NTHREADS, C::SMEM_BYTES, stream>>>(
+        mq, mk, mv, mdo, a);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   // 3. dQ accumulator -> bf16
