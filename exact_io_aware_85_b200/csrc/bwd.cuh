@@ -577,21 +577,11 @@ __global__ void __launch_bounds__(448, 1)
           const int b = t & 1;
           const int st = t % C::NST;
           if (!(ok = mbar_wait(bar_ld_full + st, (t / C::NST) & 1, abort_sh, 62))) break;
-          if (t >= 2) {
-            if (!(ok = mbar_wait(bar_dq_free + b, ((t - 2) >> 1) & 1, abort_sh, 63))) break;
-          }
           tc_fence_after();
           const uint32_t qa = q_addr + st * C::Q_TILE, da = do_addr + st * C::Q_TILE;
-          // S^T = K_j Q_i^T   (M = 128 keys, N = 64 queries, K = d)
-#pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint32_t ka = k_addr + (k >> 2) * C::KV_BOX + (k & 3) * 32;
-            const uint32_t qb = qa + (k >> 2) * C::Q_BOX + (k & 3) * 32;
-            mma_ss(tmem + C::COL_S + 64 * b, make_sdesc_sw128(ka, 16, 1024), make_sdesc_sw128(qb, 16, 1024), id_s,
-                   k > 0);
-          }
-          mma_commit(bar_s_full + b);
-          // dP^T = V_j dO_i^T
+          // dP^T = V_j dO_i^T first: its buffer was released when step t-2's
+          // gradient finished, so the tensor core has work while the dQ drain of
+          // step t-2 empties the S^T buffer
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
             const uint32_t va = v_addr + (k >> 2) * C::KV_BOX + (k & 3) * 32;
@@ -600,6 +590,19 @@ __global__ void __launch_bounds__(448, 1)
                    k > 0);
           }
           mma_commit(bar_dp_full + b);
+          if (t >= 2) {
+            if (!(ok = mbar_wait(bar_dq_free + b, ((t - 2) >> 1) & 1, abort_sh, 63))) break;
+            tc_fence_after();
+          }
+          // S^T = K_j Q_i^T   (M = 128 keys, N = 64 queries, K = d), over dQ^T(t-2)
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t ka = k_addr + (k >> 2) * C::KV_BOX + (k & 3) * 32;
+            const uint32_t qb = qa + (k >> 2) * C::Q_BOX + (k & 3) * 32;
+            mma_ss(tmem + C::COL_S + 64 * b, make_sdesc_sw128(ka, 16, 1024), make_sdesc_sw128(qb, 16, 1024), id_s,
+                   k > 0);
+          }
+          mma_commit(bar_s_full + b);
         }
         if (t >= 1) {
           const int u = t - 1;
