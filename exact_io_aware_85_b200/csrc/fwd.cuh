@@ -386,6 +386,8 @@ __global__ void __launch_bounds__(320, 1)
         // 4 independent pairs of partial row sums (packed fp32x2 adds)
         float2 rs4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         const float2 c2 = make_float2(c, c), nm2 = make_float2(neg_m, neg_m);
+        // FP8 flush counting: tiles with no masked key and no sink key need no per-key test
+        const bool plain_tile = !masked_tile && kbase >= a.n_sink;
         if constexpr (C::EB == 2) {
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
@@ -397,12 +399,19 @@ __global__ void __launch_bounds__(320, 1)
               const float p1 = ex2_approx(x.y);
               rs4[e & 3] = fadd2(rs4[e & 3], make_float2(p0, p1));
               if constexpr (FP8P) {
-                float q0, q1;
-                pk[e] = e4m3_roundtrip_bf16x2(p0 * a.p_scale, p1 * a.p_scale, q0, q1);
-                if (a.stats != nullptr && row < N) {
-                  const int k0 = kbase + h * 64 + 2 * e;
-                  if (k0 <= lim && q0 == 0.f) { if (k0 < a.n_sink) ++fl_sink; else ++fl_non; }
-                  if (k0 + 1 <= lim && q1 == 0.f) { if (k0 + 1 < a.n_sink) ++fl_sink; else ++fl_non; }
+                uint32_t nz;
+                const float2 sp = fmul2(make_float2(p0, p1), make_float2(a.p_scale, a.p_scale));
+                pk[e] = e4m3_cast_bf16x2(sp.x, sp.y, nz);
+                if (a.stats != nullptr) {
+                  if (plain_tile) {
+                    fl_non += (row < N) ? 2u - __popc(nz) : 0u;
+                  } else if (row < N) {
+                    const int k0 = kbase + h * 64 + 2 * e;
+                    const uint32_t f0 = (k0 <= lim && !(nz & 1u)) ? 1u : 0u;
+                    const uint32_t f1 = (k0 + 1 <= lim && !(nz >> 16)) ? 1u : 0u;
+                    fl_sink += (k0 < a.n_sink ? f0 : 0u) + (k0 + 1 < a.n_sink ? f1 : 0u);
+                    fl_non += (k0 < a.n_sink ? 0u : f0) + (k0 + 1 < a.n_sink ? 0u : f1);
+                  }
                 }
               } else {
                 pk[e] = pack_bf16x2(p0, p1);

@@ -344,6 +344,21 @@ __device__ __forceinline__ uint32_t e4m3_roundtrip_bf16x2(float lo, float hi, fl
   return pack_bf16x2(qlo, qhi);
 }
 
+// Same cast, returned as bf16x2 bits without leaving the integer pipes for the
+// widening: E4M3 -> f16x2 is exact and every non-zero E4M3 value is an f16
+// normal, so the bf16 bits are the f16 bits shifted right by 3 with the exponent
+// rebiased (+112 << 7); zero halves stay zero.  `nz` gets bit 0 / bit 16 set for
+// the halves that did not flush to zero.  Inputs must be >= 0.
+__device__ __forceinline__ uint32_t e4m3_cast_bf16x2(float lo, float hi, uint32_t& nz) {
+  uint16_t e;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(e) : "f"(hi), "f"(lo));
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(e));
+  const uint32_t y = (h2 >> 3) & 0x0FFF0FFFu;
+  nz = ((y + 0x7FFF7FFFu) >> 15) & 0x00010001u;
+  return y + nz * 0x3800u;
+}
+
 // Wait used only on teardown paths: bounded by time, ignores the abort flag.
 __device__ __noinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   const uint32_t a = smem_u32(bar);
