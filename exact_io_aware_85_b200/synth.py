@@ -116,5 +116,24 @@ def make_sink_inputs(B: int, H: int, N: int, d: int, delta: float, seed: int = 0
     return {"q": bf16_round(q), "k": bf16_round(k), "v": bf16_round(v)}
 
 
+def make_outlier_inputs(B: int, H: int, N: int, d: int, frac: float = 0.01, mag: float = 10.0, seed: int = 0):
+    """Q, K, V ~ N(0,1) with a fraction `frac` of entries replaced by N(0, mag^2)
+    outliers (the setting in which block-quantised FP8 attention suffers), bf16."""
+    rng = np.random.default_rng(seed)
+    out = {}
+    for name in ("q", "k", "v"):
+        x = rng.standard_normal(size=(B, H, N, d), dtype=np.float32)
+        m = rng.random(size=x.shape) < frac
+        x[m] = rng.standard_normal(size=int(m.sum()), dtype=np.float32) * np.float32(mag)
+        out[name] = bf16_round(x)
+    return out
+
+
+def random_signs(d: int, seed: int = 0) -> np.ndarray:
+    """The random +-1 diagonal of the incoherent-processing rotation (float32)."""
+    rng = np.random.default_rng(seed)
+    return np.where(rng.random(d) < 0.5, -1.0, 1.0).astype(np.float32)
+
+
 def workload_seed(name: str) -> int:
     return 1000 + list(WORKLOADS).index(name)

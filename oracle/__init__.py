@@ -18,6 +18,9 @@ Functions and the passages they follow:
 * ``attn_fwd_fp8p`` -- tile-by-tile emulation of the E4M3 P-cast with static
   scale S and forward/reverse key-tile order ("P-Cast precision in FP8
   attention", sections 1-2).
+* ``fp8_quantize`` -- E4M3 block quantisation of Q/K/V, optionally after the
+  random-sign Walsh-Hadamard rotation ("flash-attention-trading-models", section
+  "FA3", item 3: incoherent processing before block quantisation).
 * ``e4m3`` -- round to the E4M3 grid (same page: 3-bit mantissa, 448 max,
   2^-10 rounds to zero).
 * ``p_collapse_fraction``, ``collapse_threshold``, ``expected_max_normal``,
@@ -62,6 +65,8 @@ def _load():
         lib.oracle_attn_fwd_rows.argtypes = [dp, dp, dp, ip, ctypes.c_int64, dp, dp, ci, ci, ci, cd]
         lib.oracle_attn_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, ci, ci, ci, ci, ci, cd]
         lib.oracle_attn_fwd_fp8p.argtypes = [dp, dp, dp, dp, dp, ci, ci, ci, ci, ci, cd, cd, ci, ci, ci, ip]
+        lib.oracle_fp8_quantize.argtypes = [dp, dp, dp, dp, ci, ci, ci, ci]
+        lib.oracle_hadamard_rotate.argtypes = [dp, dp, dp, ctypes.c_int64, ci]
         lib.oracle_num_threads.restype = ci
         _lib = lib
     return _lib
@@ -125,6 +130,32 @@ def attn_fwd_fp8p(q, k, v, causal: bool, scale: float, S: float, kv_order: int, 
                                  float(S), int(kv_order), int(Bc), int(n_sink),
                                  counts.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)))
     return o, lse, counts
+
+
+def fp8_quantize(x, signs=None, block_rows: int = 128):
+    """Block-quantise [B,H,N,d] to E4M3 (scale = block amax / 448), optionally after
+    the rotation x -> x diag(signs) H / sqrt(d).  Returns the dequantised values
+    (code * scale, fp64, in the rotated basis when signs is given) and the scales
+    [B,H,ceil(N/block_rows)]."""
+    x = _f64(x)
+    B, H, N, d = x.shape
+    nb = (N + block_rows - 1) // block_rows
+    xq = np.empty_like(x)
+    sc = np.empty((B, H, nb), dtype=np.float64)
+    sg = None if signs is None else _f64(signs)
+    _load().oracle_fp8_quantize(_ptr(x), None if sg is None else _ptr(sg), _ptr(xq), _ptr(sc), B * H, N, d,
+                                int(block_rows))
+    return xq, sc
+
+
+def hadamard_rotate(x, signs):
+    """x diag(signs) H / sqrt(d) applied to every row (last axis) of x, fp64."""
+    x = _f64(x)
+    d = x.shape[-1]
+    y = np.empty_like(x)
+    sg = _f64(signs)
+    _load().oracle_hadamard_rotate(_ptr(x.reshape(-1)), _ptr(sg), _ptr(y.reshape(-1)), x.size // d, d)
+    return y
 
 
 def e4m3(x) -> np.ndarray:

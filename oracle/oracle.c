@@ -264,6 +264,70 @@ void oracle_attn_fwd_fp8p(const double* Q, const double* K, const double* V, dou
   counts[3] = c3;
 }
 
+/* ------------------------------------------------------------------------- */
+/* FP8 operands with incoherent processing ("flash-attention-trading-models", */
+/* section "FA3", item 3): rows are multiplied by a random orthogonal matrix   */
+/* (random signs, then the normalised Walsh-Hadamard matrix) before block     */
+/* quantisation to E4M3, which spreads an outlier's magnitude over the row.   */
+/* ------------------------------------------------------------------------- */
+/* y = x diag(signs) H / sqrt(d) for one row, H the Sylvester Hadamard matrix,
+ * H[i][j] = (-1)^popcount(i & j); written as the definition, O(d^2). */
+static void rotate_row(const double* x, const double* signs, double* y, int d) {
+  const double norm = 1.0 / sqrt((double)d);
+  for (int j = 0; j < d; ++j) {
+    double acc = 0.0;
+    for (int i = 0; i < d; ++i) {
+      const int par = __builtin_popcount((unsigned)(i & j)) & 1;
+      acc += (par ? -1.0 : 1.0) * signs[i] * x[i];
+    }
+    y[j] = acc * norm;
+  }
+}
+
+/* The rotation alone, for `rows` rows of length d. */
+void oracle_hadamard_rotate(const double* X, const double* signs, double* Y, int64_t rows, int d) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r) rotate_row(X + r * d, signs, Y + r * d, d);
+}
+
+/* Quantise [BH, N, d] to E4M3 with one scale per block of `block_rows` rows
+ * of each (b,h) (block_rows >= N gives one scale per head).  signs == NULL
+ * means no rotation.  Outputs: xq (the dequantised values code * scale, fp64)
+ * and scales [BH, ceil(N/block_rows)] with scale = amax / 448 (1 for an
+ * all-zero block). */
+void oracle_fp8_quantize(const double* X, const double* signs, double* XQ, double* scales, int BH, int N, int d,
+                         int block_rows) {
+  const int nb = (N + block_rows - 1) / block_rows;
+#pragma omp parallel
+  {
+    double* y = (double*)malloc(sizeof(double) * (size_t)d * (size_t)block_rows);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t t = 0; t < (int64_t)BH * nb; ++t) {
+      const int64_t bh = t / nb;
+      const int blk = (int)(t % nb);
+      const int r0 = blk * block_rows;
+      int r1 = r0 + block_rows;
+      if (r1 > N) r1 = N;
+      double amax = 0.0;
+      for (int r = r0; r < r1; ++r) {
+        const double* x = X + (bh * N + r) * (int64_t)d;
+        double* yr = y + (int64_t)(r - r0) * d;
+        if (signs) rotate_row(x, signs, yr, d);
+        else for (int c = 0; c < d; ++c) yr[c] = x[c];
+        for (int c = 0; c < d; ++c) if (fabs(yr[c]) > amax) amax = fabs(yr[c]);
+      }
+      const double sc = amax > 0.0 ? amax / 448.0 : 1.0;
+      scales[bh * nb + blk] = sc;
+      for (int r = r0; r < r1; ++r) {
+        const double* yr = y + (int64_t)(r - r0) * d;
+        double* q = XQ + (bh * N + r) * (int64_t)d;
+        for (int c = 0; c < d; ++c) q[c] = oracle_e4m3(yr[c] / sc) * sc;
+      }
+    }
+    free(y);
+  }
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();
