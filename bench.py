@@ -150,7 +150,7 @@ def device_inputs(w: synth.Workload, seed: int):
     g = torch.Generator(device="cuda")
     g.manual_seed(seed)
     shape = (w.B, w.H, w.N, w.d)
-    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
     q = torch.randn(shape, generator=g, device="cuda", dtype=torch.float32).to(dt)
     k = torch.randn(shape, generator=g, device="cuda", dtype=torch.float32).to(dt)
     v = torch.randn(shape, generator=g, device="cuda", dtype=torch.float32).to(dt)
@@ -216,7 +216,9 @@ METRIC = "attention fwd/bwd TFLOP/s at 1 B200 and % of dense BF16/FP8 tensor pea
 
 def config_of(w, ws):
     what = ("forward + backward (dQ, dK, dV from the saved LSE)" if w.backward else
-            "FP8 P-cast forward, S=256, forward key order, sink Delta=8" if w.sink else "forward (O + LSE)")
+            "FP8 P-cast forward, S=256, forward key order, sink Delta=8" if w.sink else
+            "E4M3 forward (Hadamard-rotated block-quantised Q/K, per-head V, P-cast S=256)" if w.dtype == "fp8"
+            else "forward (O + LSE)")
     return {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} {w.dtype} "
                         f"{'causal' if w.causal else 'non-causal'} {what}",
             "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal, "parallelism": f"replicas x{ws}",
@@ -268,6 +270,26 @@ def main():
 
         def run():
             fa.fa_fwd_fp8p(q, k, v, o, lse, w.causal, w.scale, 256.0, 0, stats, 4)
+    elif w.dtype == "fp8":
+        # E4M3 operands prepared once (quantisation with the random-sign Hadamard
+        # rotation, outside the timed step); the step is the FP8 attention kernel
+        nb = (w.N + 127) // 128
+        q8, k8, v8 = (torch.empty(q.shape, dtype=torch.uint8, device="cuda") for _ in range(3))
+        sq = torch.empty((w.B, w.H, nb), dtype=torch.float32, device="cuda")
+        sk = torch.empty_like(sq)
+        sv = torch.empty((w.B, w.H), dtype=torch.float32, device="cuda")
+        signs = torch.from_numpy(synth.random_signs(w.d, seed=synth.workload_seed(w.name))).cuda()
+        fa.fa_fp8_quantize(q, k, v, signs, q8, k8, v8, sq, sk, sv)
+        qz0 = torch.cuda.Event(enable_timing=True)
+        qz1 = torch.cuda.Event(enable_timing=True)
+        qz0.record()
+        fa.fa_fp8_quantize(q, k, v, signs, q8, k8, v8, sq, sk, sv)
+        qz1.record()
+        torch.cuda.synchronize()
+        quant_ms = qz0.elapsed_time(qz1)
+
+        def run():
+            fa.fa_fwd_fp8(q8, k8, v8, sq, sk, sv, o, lse, w.causal, w.scale, 256.0, 0)
     elif w.dtype == "bf16":
         def run():
             fa.fa_fwd(q, k, v, o, lse, w.causal, w.scale)
@@ -323,6 +345,8 @@ def main():
         v.copy_(hv, non_blocking=True)
         if w.backward:
             do.copy_(hdo, non_blocking=True)
+        if w.dtype == "fp8":  # end to end includes the quantisation of the fresh inputs
+            fa.fa_fp8_quantize(q, k, v, signs, q8, k8, v8, sq, sk, sv)
         run()
         if w.backward:
             hdq.copy_(dq, non_blocking=True)
@@ -349,10 +373,17 @@ def main():
         h2d += do.numel() * do.element_size()
 
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_note = f"{peak_src} bf16 burst (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback 1590 TFLOP/s"
+    if w.dtype == "fp8":
+        # no measured FP8 peak on this machine: the measured bf16 peak x the nominal 2x FP8 ratio
+        peak *= 2.0
+        peak_note = f"{peak_src} bf16 burst x 2 (nominal FP8/BF16 ratio)"
     if w.backward:
         kernel_name = "training step: fa_fwd_kernel<bf16,%d> + fa_bwd (pre, main, post)" % w.d
     elif w.sink:
         kernel_name = "fa_fwd_kernel<bf16,%d,FP8P>" % w.d
+    elif w.dtype == "fp8":
+        kernel_name = "fa_fwd_kernel<e4m3,%d> (kind::f8f6f4)" % w.d
     else:
         kernel_name = "fa_fwd_kernel<%s,%d>" % ("bf16" if w.dtype == "bf16" else "f32/tf32", w.d)
     achieved = flops / (step_ms_local * 1e-3) / 1e12
@@ -364,15 +395,14 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "vs_baseline": None, "dtype": {"bf16": "bf16", "f32": "f32", "fp8": "e4m3"}[w.dtype], "data": "synthetic",
             "config": config_of(w, ws),
             "tokens_per_s": ws * w.B * w.N / (step_ms * 1e-3),
             "pct_of_peak": {"measured_bf16_burst": achieved / peak,
                             "measured_bf16_sustained": achieved / float(peaks.get("bf16_tflops_sustained", 1390.0)),
                             "datasheet_bf16_2250": achieved / 2250.0},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)"
-                         if peak_src == "measured" else "fallback 1590 TFLOP/s",
+                         "frac": achieved / peak, "peak_source": peak_note,
                          "traffic": traffic, "kernel": kernel_name,
                          "launch_ms": {"median": statistics.median(launch_ms), "min": min(launch_ms),
                                        "mean": step_ms_local}},
@@ -381,6 +411,8 @@ def main():
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": args.steps * launches_per_step,
         }
+        if w.dtype == "fp8":
+            line["fp8_quantize_ms"] = quant_ms
         if ws == 1 and not args.no_cpu_baseline:
             cb = cpu_baseline(w)
             cb.pop("seconds", None)

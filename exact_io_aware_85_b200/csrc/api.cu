@@ -15,6 +15,7 @@
 #include "sm100.cuh"
 #include "fwd.cuh"
 #include "bwd.cuh"
+#include "fp8.cuh"
 
 namespace fa {
 // Self-test of the failure path: waits on an mbarrier that nothing will ever
@@ -91,10 +92,12 @@ int check_common(const void* q, const void* k, const void* v, const void* o, con
 
 template <typename T, int D, bool FP8P>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int causal,
-               float scale, float S, int kv_order, unsigned long long* stats, int n_sink, cudaStream_t stream) {
+               float scale, float S, int kv_order, unsigned long long* stats, int n_sink, cudaStream_t stream,
+               const float* sq = nullptr, const float* sk = nullptr, const float* sv = nullptr) {
   using C = fa::FwdCfg<T, D, FP8P>;
-  constexpr CUtensorMapDataType dt =
-      sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  constexpr CUtensorMapDataType dt = sizeof(T) == 2   ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                     : sizeof(T) == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                                      : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   const int BH = B * H;
   CUtensorMap mq, mk, mv;
   int st;
@@ -102,7 +105,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   if ((st = encode_qkv_map(&mk, k, dt, sizeof(T), D, N, BH)) != FA_OK) return st;
   // fp32 V feeds the tf32 MMA as an MN-major operand, which needs the 32-byte-atom swizzle
   if ((st = encode_qkv_map(&mv, v, dt, sizeof(T), D, N, BH,
-                           sizeof(T) == 2 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B)) != FA_OK)
+                           sizeof(T) == 4 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
     return st;
   fa::FwdArgs a;
   a.o = o;
@@ -116,6 +119,10 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   a.kv_order = kv_order;
   a.stats = stats;
   a.n_sink = n_sink;
+  a.sq = sq;
+  a.sk = sk;
+  a.sv = sv;
+  a.nqb = (N + 127) / 128;
   auto kern = fa::fa_fwd_kernel<T, D, FP8P>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -261,6 +268,61 @@ int fa_fwd_fp8p(const void* q, const void* k, const void* v, void* o, float* lse
   if (d == 64)
     return launch_fwd<__nv_bfloat16, 64, true>(q, k, v, o, lse, B, H, N, causal, scale, S, kv_order, stats, n_sink, s);
   return launch_fwd<__nv_bfloat16, 128, true>(q, k, v, o, lse, B, H, N, causal, scale, S, kv_order, stats, n_sink, s);
+}
+
+int fa_fp8_quantize(const void* q, const void* k, const void* v, const float* signs, void* q8, void* k8, void* v8,
+                    float* sq, float* sk, float* sv, int B, int H, int N, int d, void* stream) {
+  if (!q || !k || !v || !q8 || !k8 || !v8 || !sq || !sk || !sv) return FA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H * N * d >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q8) || !aligned16(k8) || !aligned16(v8))
+    return FA_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(sq) | reinterpret_cast<uintptr_t>(sk) | reinterpret_cast<uintptr_t>(sv) |
+       reinterpret_cast<uintptr_t>(signs)) & 3u)
+    return FA_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  fa::Fp8QuantArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.v = static_cast<const __nv_bfloat16*>(v);
+  a.signs = signs;
+  a.q8 = static_cast<uint8_t*>(q8);
+  a.k8 = static_cast<uint8_t*>(k8);
+  a.v8 = static_cast<uint8_t*>(v8);
+  a.sq = sq;
+  a.sk = sk;
+  a.sv = sv;
+  a.N = N;
+  a.nblk = (N + 127) / 128;
+  fa::fa_fp8_v_clear_kernel<<<(BH + 255) / 256, 256, 0, s>>>(sv, BH);
+  const dim3 grid(a.nblk, BH, 3);
+  const long long nvec = static_cast<long long>(BH) * N * (d / 8);
+  if (d == 64) {
+    fa::fa_fp8_qk_quant_kernel<64><<<grid, 128, 0, s>>>(a);
+    fa::fa_fp8_v_quant_kernel<64><<<static_cast<unsigned>((nvec + 255) / 256), 256, 0, s>>>(a, nvec);
+  } else {
+    fa::fa_fp8_qk_quant_kernel<128><<<grid, 128, 0, s>>>(a);
+    fa::fa_fp8_v_quant_kernel<128><<<static_cast<unsigned>((nvec + 255) / 256), 256, 0, s>>>(a, nvec);
+  }
+  fa::fa_fp8_v_scale_kernel<<<(BH + 255) / 256, 256, 0, s>>>(sv, BH);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return FA_OK;
+}
+
+int fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* sq, const float* sk, const float* sv,
+               void* o, float* lse, int B, int H, int N, int d, int causal, float scale, float S, int kv_order,
+               void* stream) {
+  int st = check_common(q8, k8, v8, o, lse, B, H, N, d, scale);
+  if (st != FA_OK) return st;
+  if (d != 128) return FA_ERR_UNSUPPORTED;  // E4M3 rows of 64 bytes would need the 64-byte swizzle
+  if (!sq || !sk || !sv) return FA_ERR_INVALID_ARG;
+  if (!(std::isfinite(S) && S > 0.f)) return FA_ERR_INVALID_ARG;
+  if (kv_order != 0 && kv_order != 1) return FA_ERR_INVALID_ARG;
+  return launch_fwd<uint8_t, 128, true>(q8, k8, v8, o, lse, B, H, N, causal, scale, S, kv_order, nullptr, 0,
+                                        static_cast<cudaStream_t>(stream), sq, sk, sv);
 }
 
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {

@@ -30,6 +30,8 @@
 // key tiles wholly in the future of a Q tile are never loaded or multiplied;
 // the diagonal tile and the ragged last key tile are masked element-wise.
 #pragma once
+#include <type_traits>
+
 #include "sm100.cuh"
 
 namespace fa {
@@ -46,6 +48,12 @@ struct ElemTraits<float> {
   static constexpr int kBytes = 4;
   static constexpr uint32_t kFmt = kFmtTF32;
 };
+// E4M3 codes (the full FP8 forward): kind::f8f6f4 MMAs
+template <>
+struct ElemTraits<uint8_t> {
+  static constexpr int kBytes = 1;
+  static constexpr uint32_t kFmt = kFmtE4M3;
+};
 
 struct FwdArgs {
   void* o;
@@ -59,6 +67,11 @@ struct FwdArgs {
   int kv_order;      // 0: key tiles 0..T-1, 1: T-1..0
   unsigned long long* stats;
   int n_sink;
+  // full FP8 operands only: dequantisation scales of the E4M3 codes
+  const float* sq;  // [BH, nqb] per 128-row block of Q
+  const float* sk;  // [BH, nqb] per 128-row block of K
+  const float* sv;  // [BH] per head of V
+  int nqb;          // ceil(N / 128)
 };
 
 template <typename T, int D, bool FP8P>
@@ -211,6 +224,8 @@ __global__ void __launch_bounds__(320, 1)
           if (!leader) continue;
           if constexpr (C::EB == 2)
             mma_ss(tmem + (i ? C::COL_S1 : C::COL_S0), ad, bd, idesc_s, k > 0);
+          else if constexpr (C::EB == 1)
+            mma_ss_f8(tmem + (i ? C::COL_S1 : C::COL_S0), ad, bd, idesc_s, k > 0);
           else
             mma_ss_tf32(tmem + (i ? C::COL_S1 : C::COL_S0), ad, bd, idesc_s, k > 0);
         }
@@ -222,14 +237,16 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t ocol = tmem + (i ? C::COL_O1 : C::COL_O0);
 #pragma unroll
         for (int k = 0; k < C::NK_PV; ++k) {
-          // V is the MN-major B operand: 128B swizzle (bf16) or the 32-byte-atom
+          // V is the MN-major B operand: 128B swizzle (bf16, E4M3) or the 32-byte-atom
           // 128B swizzle (tf32, whose only MN-major layout), K rows 128 B apart.
-          const uint64_t bd = C::EB == 2 ? make_sdesc_sw128(va + k * C::KSTEP * 128, C::BOX_BYTES, 1024)
-                                         : make_sdesc_sw128_32b(va + k * C::KSTEP * 128, C::BOX_BYTES, 512);
+          const uint64_t bd = C::EB == 4 ? make_sdesc_sw128_32b(va + k * C::KSTEP * 128, C::BOX_BYTES, 512)
+                                         : make_sdesc_sw128(va + k * C::KSTEP * 128, C::BOX_BYTES, 1024);
           const uint32_t acc = (pv_count[i] > 0 || k > 0) ? 1u : 0u;
           if (!leader) continue;
           if constexpr (C::EB == 2)
             mma_ts(ocol, pcol + k * 8, bd, idesc_pv, acc);
+          else if constexpr (C::EB == 1)
+            mma_ts_f8(ocol, pcol + k * 8, bd, idesc_pv, acc);
           else
             mma_ts_tf32(ocol, pcol + k * 8, bd, idesc_pv, acc);
         }
@@ -325,7 +342,9 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t tO = tmem + lane_base + (i ? C::COL_O1 : C::COL_O0);
     const int kv_end = i ? kv_end1 : kv_end0;
     const int qt = qt0 + i;
-    const float c = a.scale_log2;
+    // E4M3 operands carry block scales: the score factor of tile j is
+    // scale*log2(e) * sq[query block] * sk[key block j]
+    const float c_base = C::EB == 1 ? a.scale_log2 * a.sq[static_cast<size_t>(bh) * a.nqb + qt] : a.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
     uint32_t fl_sink = 0, fl_non = 0;
     int cnt = 0;
@@ -334,6 +353,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int t = 0; t < n_steps; ++t) {
         const int j = rev ? n_steps - 1 - t : t;
         if (j >= kv_end) continue;
+        const float c = C::EB == 1 ? c_base * a.sk[static_cast<size_t>(bh) * a.nqb + j] : c_base;
         if (!(ok = mbar_wait(&bar_s[i], cnt & 1, &abort_sh, 10 + i))) break;
         tc_fence_after();
         float sv[128];
@@ -388,7 +408,25 @@ __global__ void __launch_bounds__(320, 1)
         const float2 c2 = make_float2(c, c), nm2 = make_float2(neg_m, neg_m);
         // FP8 flush counting: tiles with no masked key and no sink key need no per-key test
         const bool plain_tile = !masked_tile && kbase >= a.n_sink;
-        if constexpr (C::EB == 2) {
+        if constexpr (C::EB == 1) {
+          // P' = E4M3(S p), four codes per 32-bit TMEM column (the PV MMA's A operand)
+          uint32_t pk[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float2 x01 = ffma2(make_float2(sv[4 * e], sv[4 * e + 1]), c2, nm2);
+            const float2 x23 = ffma2(make_float2(sv[4 * e + 2], sv[4 * e + 3]), c2, nm2);
+            const float2 p01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
+            const float2 p23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
+            rs4[e & 3] = fadd2(rs4[e & 3], fadd2(p01, p23));
+            const float2 s01 = fmul2(p01, make_float2(a.p_scale, a.p_scale));
+            const float2 s23 = fmul2(p23, make_float2(a.p_scale, a.p_scale));
+            uint16_t lo, hi;
+            asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(s01.y), "f"(s01.x));
+            asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(s23.y), "f"(s23.x));
+            pk[e] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+          }
+          tmem_st32(tS, pk);
+        } else if constexpr (C::EB == 2) {
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             uint32_t pk[32];
@@ -464,15 +502,17 @@ __global__ void __launch_bounds__(320, 1)
       if (ok) ok = mbar_wait(&bar_o[i], 0, &abort_sh, 12 + i);
       if (ok) {
         tc_fence_after();
-        const float inv = 1.0f / (l_run * a.p_scale);
-        T* orow = reinterpret_cast<T*>(a.o) + (static_cast<size_t>(bh) * N + row) * D;
+        const float inv = (C::EB == 1 ? a.sv[bh] : 1.0f) / (l_run * a.p_scale);
+        // output: fp32 for fp32 inputs, bf16 otherwise (also for E4M3 operands)
+        using OutT = typename std::conditional<C::EB == 4, float, __nv_bfloat16>::type;
+        OutT* orow = reinterpret_cast<OutT*>(a.o) + (static_cast<size_t>(bh) * N + row) * D;
 #pragma unroll
         for (int ch = 0; ch < D / 32; ++ch) {
           uint32_t ov[32];
           tmem_ld32(tO + ch * 32, ov);
           tmem_wait_ld();
           if (row < N) {
-            if constexpr (C::EB == 2) {
+            if constexpr (C::EB != 4) {
               uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
 #pragma unroll
               for (int v4 = 0; v4 < 4; ++v4) {

@@ -121,3 +121,22 @@ def fa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, causal: bool, scale: float, 
     B, H, N, d = _dims(q)
     _check(lib.fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
                               B, H, N, d, int(causal), float(scale), _stream(stream)), "fa_bwd_noalloc")
+
+
+lib.fa_fp8_quantize.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _vp]
+lib.fa_fwd_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _cf, _cf, _ci, _vp]
+
+
+def fa_fp8_quantize(q, k, v, signs, q8, k8, v8, sq, sk, sv, stream=None) -> None:
+    """E4M3 codes (uint8 tensors) and scales for fa_fwd_fp8; signs: fp32 [d] or None."""
+    B, H, N, d = _dims(q)
+    _check(lib.fa_fp8_quantize(_ptr(q), _ptr(k), _ptr(v), _ptr(signs), _ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq),
+                               _ptr(sk), _ptr(sv), B, H, N, d, _stream(stream)), "fa_fp8_quantize")
+
+
+def fa_fwd_fp8(q8, k8, v8, sq, sk, sv, o, lse, causal: bool, scale: float, S: float = 256.0, kv_order: int = 0,
+               stream=None) -> None:
+    """Forward on E4M3 operands; o is bf16 [B,H,N,d]."""
+    B, H, N, d = _dims(q8)
+    _check(lib.fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq), _ptr(sk), _ptr(sv), _ptr(o), _ptr(lse), B, H, N,
+                          d, int(causal), float(scale), float(S), int(kv_order), _stream(stream)), "fa_fwd_fp8")

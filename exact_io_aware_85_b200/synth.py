@@ -30,7 +30,7 @@ class Workload:
     H: int
     N: int
     d: int
-    dtype: str  # "bf16" or "f32"
+    dtype: str  # "bf16", "f32", or "fp8" (bf16 inputs quantised to E4M3)
     causal: bool
     backward: bool = False
     sink: bool = False
@@ -55,6 +55,8 @@ WORKLOADS = {
     "prefill": Workload("prefill", 4, 32, 8192, 128, "bf16", True),
     "train": Workload("train", 2, 16, 4096, 128, "bf16", True, backward=True),
     "sink": Workload("sink", 1, 32, 16384, 128, "bf16", False, sink=True),
+    # the prefill shape on E4M3 operands (full FP8 forward with incoherent processing)
+    "prefill_fp8": Workload("prefill_fp8", 4, 32, 8192, 128, "fp8", True),
 }
 
 SINK_DELTAS = (0.0, 2.0, 4.0, 6.0, 7.0, 8.0, 10.0, 12.0)

@@ -112,6 +112,30 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
 int fa_fwd_fp8p(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
                 int causal, float scale, float S, int kv_order, unsigned long long* stats, int n_sink, void* stream);
 
+/* FP8 operands for fa_fwd_fp8 ("flash-attention-trading-models", section "FA3",
+ * item 3: FP8 with incoherent processing).  Quantises bf16 q, k, v [B,H,N,d]
+ * to E4M3 codes (round to nearest even, saturating):
+ *  - q and k, one scale per block of 128 rows of each (b,h), after the optional
+ *    rotation x -> x diag(signs) H / sqrt(d) (H the Sylvester Walsh-Hadamard
+ *    matrix; signs = NULL skips it): the caller draws the d random signs (+-1,
+ *    fp32 device array).  The rotation leaves q k^T unchanged and spreads
+ *    outliers, which is what lowers the quantisation error;
+ *  - v, one scale per head, never rotated.
+ * Outputs (caller-owned device memory): q8, k8, v8 uint8 [B,H,N,d] E4M3 codes;
+ * sq, sk fp32 [B,H,ceil(N/128)] and sv fp32 [B,H] dequantisation scales
+ * (block amax / 448, 1 for an all-zero block).  d in {64, 128}. */
+int fa_fp8_quantize(const void* q, const void* k, const void* v, const float* signs, void* q8, void* k8, void* v8,
+                    float* sq, float* sk, float* sv, int B, int H, int N, int d, void* stream);
+
+/* Forward on E4M3 operands from fa_fp8_quantize: S = (q8 k8^T)(sq sk) scale on
+ * the kind::f8f6f4 tensor cores, the online softmax in fp32, P' = E4M3(S_p p)
+ * (static scale S_p, key-tile order kv_order as in fa_fwd_fp8p), O += P' v8 on
+ * the tensor cores, and O = acc * sv / (S_p * l) -> bf16 [B,H,N,d]; lse fp32
+ * [B,H,N] of the quantised scores.  d = 128 only. */
+int fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* sq, const float* sk, const float* sv,
+               void* o, float* lse, int B, int H, int N, int d, int causal, float scale, float S, int kv_order,
+               void* stream);
+
 /* Human-readable name of an fa_status code. */
 const char* fa_status_string(int status);
 
