@@ -15,6 +15,8 @@ Functions and the passages they follow:
   memoria"; "FlashAttention (IT)", "Problematica dell'attention standard").
 * ``attn_bwd`` -- derivatives of that definition (the pages only say the
   backward recomputes the scores, "Pase hacia atras"; the calculus is standard).
+* ``attn_fwd_gqa`` / ``attn_bwd_gqa`` -- grouped-query / multi-query attention as
+  attention over key/value heads repeated across each query-head group.
 * ``attn_fwd_fp8p`` -- tile-by-tile emulation of the E4M3 P-cast with static
   scale S and forward/reverse key-tile order ("P-Cast precision in FP8
   attention", sections 1-2).
@@ -116,6 +118,27 @@ def attn_bwd(q, k, v, do, causal: bool, scale: float):
     _load().oracle_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d,
                             int(causal), float(scale))
     return dq, dk, dv
+
+
+def attn_fwd_gqa(q, k, v, causal: bool, scale: float):
+    """Grouped-query attention: q [B,Hq,N,d], k and v [B,Hkv,N,d] with Hq a multiple
+    of Hkv; query head h attends with key/value head h // (Hq/Hkv) (multi-query
+    attention is Hkv = 1).  By definition this is attention with every key/value
+    head repeated for the query heads of its group ("FlashAttention for Scalable
+    Vector Architectures", "Metodologia": the shared KV head; "FlashAttention
+    (IT)", "FlashAttention-2": Multi-Query Attention)."""
+    g = q.shape[1] // k.shape[1]
+    return attn_fwd(q, np.repeat(_f64(k), g, axis=1), np.repeat(_f64(v), g, axis=1), causal, scale)
+
+
+def attn_bwd_gqa(q, k, v, do, causal: bool, scale: float):
+    """Gradients of grouped-query attention: dK and dV of a key/value head are the
+    sums of the repeated heads' gradients over its group."""
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    g = Hq // Hkv
+    dq, dk, dv = attn_bwd(q, np.repeat(_f64(k), g, axis=1), np.repeat(_f64(v), g, axis=1), do, causal, scale)
+    return dq, dk.reshape(B, Hkv, g, N, d).sum(axis=2), dv.reshape(B, Hkv, g, N, d).sum(axis=2)
 
 
 def attn_fwd_fp8p(q, k, v, causal: bool, scale: float, S: float, kv_order: int, Bc: int = 128, n_sink: int = 4):
