@@ -93,7 +93,8 @@ int check_common(const void* q, const void* k, const void* v, const void* o, con
 template <typename T, int D, bool FP8P>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int causal,
                float scale, float S, int kv_order, unsigned long long* stats, int n_sink, cudaStream_t stream,
-               const float* sq = nullptr, const float* sk = nullptr, const float* sv = nullptr) {
+               const float* sq = nullptr, const float* sk = nullptr, const float* sv = nullptr, int Hkv = 0) {
+  if (Hkv <= 0) Hkv = H;
   using C = fa::FwdCfg<T, D, FP8P>;
   constexpr CUtensorMapDataType dt = sizeof(T) == 2   ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                      : sizeof(T) == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
@@ -102,9 +103,9 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   CUtensorMap mq, mk, mv;
   int st;
   if ((st = encode_qkv_map(&mq, q, dt, sizeof(T), D, N, BH)) != FA_OK) return st;
-  if ((st = encode_qkv_map(&mk, k, dt, sizeof(T), D, N, BH)) != FA_OK) return st;
+  if ((st = encode_qkv_map(&mk, k, dt, sizeof(T), D, N, B * Hkv)) != FA_OK) return st;
   // fp32 V feeds the tf32 MMA as an MN-major operand, which needs the 32-byte-atom swizzle
-  if ((st = encode_qkv_map(&mv, v, dt, sizeof(T), D, N, BH,
+  if ((st = encode_qkv_map(&mv, v, dt, sizeof(T), D, N, B * Hkv,
                            sizeof(T) == 4 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
     return st;
   fa::FwdArgs a;
@@ -123,6 +124,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   a.sk = sk;
   a.sv = sv;
   a.nqb = (N + 127) / 128;
+  a.group = H / Hkv;
   auto kern = fa::fa_fwd_kernel<T, D, FP8P>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -136,9 +138,11 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
 template <int D>
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse, void* dq,
                void* dk, void* dv, int B, int H, int N, int causal, float scale, void* workspace,
-               cudaStream_t stream) {
+               cudaStream_t stream, int Hkv = 0) {
   using C = fa::BwdCfg<D>;
+  if (Hkv <= 0) Hkv = H;
   const int BH = B * H;
+  const int BHkv = B * Hkv;
   const int n_tiles = (N + 127) / 128;
   const int npad = n_tiles * 128;
   float* lse2 = static_cast<float*>(workspace);
@@ -148,8 +152,8 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   int st;
   const auto dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   if ((st = encode_qkv_map(&mq, q, dt, 2, D, N, BH)) != FA_OK) return st;
-  if ((st = encode_qkv_map(&mk, k, dt, 2, D, N, BH)) != FA_OK) return st;
-  if ((st = encode_qkv_map(&mv, v, dt, 2, D, N, BH)) != FA_OK) return st;
+  if ((st = encode_qkv_map(&mk, k, dt, 2, D, N, BHkv)) != FA_OK) return st;
+  if ((st = encode_qkv_map(&mv, v, dt, 2, D, N, BHkv)) != FA_OK) return st;
   if ((st = encode_qkv_map(&mdo, dO, dt, 2, D, N, BH)) != FA_OK) return st;
   // 1. D, LSE*log2(e), zeroed dQ accumulator
   const long long rows = static_cast<long long>(BH) * npad;
@@ -170,6 +174,8 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   a.Npad = npad;
   a.BH = BH;
   a.n_tiles = n_tiles;
+  a.group = H / Hkv;
+  a.BHkv = BHkv;
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.causal = causal ? 1 : 0;
@@ -182,13 +188,13 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     auto kern = fa::fa_bwd_main_q64_kernel;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, CQ::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e);
-    kern<<<static_cast<unsigned>(static_cast<long long>(n_tiles) * BH), CQ::NTHREADS, CQ::SMEM_BYTES, stream>>>(
+    kern<<<static_cast<unsigned>(static_cast<long long>(n_tiles) * BHkv), CQ::NTHREADS, CQ::SMEM_BYTES, stream>>>(
         mq64, mk, mv, mdo64, a);
   } else {
     auto kern = fa::fa_bwd_main_kernel<D>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e);
-    kern<<<static_cast<unsigned>(static_cast<long long>(n_tiles) * BH), C::NTHREADS, C::SMEM_BYTES, stream>>>(
+    kern<<<static_cast<unsigned>(static_cast<long long>(n_tiles) * BHkv), C::NTHREADS, C::SMEM_BYTES, stream>>>(
         mq, mk, mv, mdo, a);
   }
   e = cudaGetLastError();
@@ -268,6 +274,34 @@ int fa_fwd_fp8p(const void* q, const void* k, const void* v, void* o, float* lse
   if (d == 64)
     return launch_fwd<__nv_bfloat16, 64, true>(q, k, v, o, lse, B, H, N, causal, scale, S, kv_order, stats, n_sink, s);
   return launch_fwd<__nv_bfloat16, 128, true>(q, k, v, o, lse, B, H, N, causal, scale, S, kv_order, stats, n_sink, s);
+}
+
+int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv, int N, int d,
+               int causal, float scale, void* stream) {
+  int st = check_common(q, k, v, o, lse, B, H, N, d, scale);
+  if (st != FA_OK) return st;
+  if (H_kv < 1 || H % H_kv != 0) return FA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 64)
+    return launch_fwd<__nv_bfloat16, 64, false>(q, k, v, o, lse, B, H, N, causal, scale, 1.f, 0, nullptr, 0, s,
+                                                nullptr, nullptr, nullptr, H_kv);
+  return launch_fwd<__nv_bfloat16, 128, false>(q, k, v, o, lse, B, H, N, causal, scale, 1.f, 0, nullptr, 0, s,
+                                               nullptr, nullptr, nullptr, H_kv);
+}
+
+int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse, void* dq,
+               void* dk, void* dv, int B, int H, int H_kv, int N, int d, int causal, float scale, void* workspace,
+               size_t workspace_bytes, void* stream) {
+  int st = check_common(q, k, v, o, lse, B, H, N, d, scale);
+  if (st != FA_OK) return st;
+  if (H_kv < 1 || H % H_kv != 0) return FA_ERR_INVALID_ARG;
+  if (!dO || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
+  if (!aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return FA_ERR_ALIGNMENT;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FA_ERR_ALIGNMENT;
+  if (workspace_bytes < fa_bwd_workspace_bytes(B, H, N, d)) return FA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_bwd<64>(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, causal, scale, workspace, s, H_kv)
+                 : launch_bwd<128>(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, causal, scale, workspace, s, H_kv);
 }
 
 int fa_fp8_quantize(const void* q, const void* k, const void* v, const float* signs, void* q8, void* k8, void* v8,

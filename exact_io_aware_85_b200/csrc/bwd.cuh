@@ -107,6 +107,8 @@ struct BwdArgs {
   const float* dvec;  // [BH, Npad] D, 0 on padding rows
   float* dq_acc;      // [BH, Npad, d]
   int N, Npad, BH, n_tiles;
+  int group;         // query heads per key/value head (1 = multi-head attention)
+  int BHkv;          // batch * key/value heads
   float scale;       // softmax scale
   float scale_log2;  // scale * log2(e)
   int causal;
@@ -172,10 +174,14 @@ __global__ void __launch_bounds__(448, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int N = a.N;
-  const int bh = blockIdx.x % a.BH;
-  const int j = blockIdx.x / a.BH;  // key tile; j = 0 (the longest walk when causal) first
+  const int bh_kv = blockIdx.x % a.BHkv;  // key/value head
+  const int j = blockIdx.x / a.BHkv;      // key tile; j = 0 (the longest walk when causal) first
   const int i0 = a.causal ? j : 0;
-  const int steps = a.n_tiles - i0;
+  const int spq = a.n_tiles - i0;         // query tiles per query head
+  const int steps = spq * a.group;        // the walk covers every query head of the group
+  // step t -> (query head, query tile)
+  auto step_head = [&](int t) { return bh_kv * a.group + t / spq; };
+  auto step_tile = [&](int t) { return i0 + t % spq; };
 
   // the swizzled TMA/UMMA layouts need a 1024-byte aligned base
   if ((smem_u32(smem) & 1023u) != 0) {
@@ -217,21 +223,21 @@ __global__ void __launch_bounds__(448, 1)
       tma_prefetch_desc(&tmDO);
       mbar_arrive_expect_tx(bar_kv, 2 * C::TILE);
       for (int b = 0; b < C::NBOX; ++b) {
-        tma_load_3d(smem + C::OFF_K + b * C::BOX, &tmK, bar_kv, b * 64, j * 128, bh);
-        tma_load_3d(smem + C::OFF_V + b * C::BOX, &tmV, bar_kv, b * 64, j * 128, bh);
+        tma_load_3d(smem + C::OFF_K + b * C::BOX, &tmK, bar_kv, b * 64, j * 128, bh_kv);
+        tma_load_3d(smem + C::OFF_V + b * C::BOX, &tmV, bar_kv, b * 64, j * 128, bh_kv);
       }
       int t = 0;
       for (; t < steps; ++t) {
-        const int i = i0 + t;
+        const int i = step_tile(t), hq = step_head(t);
         const int s = t & 1;
         const uint32_t ph = (t >> 1) & 1;
         if (!mbar_wait(bar_ld_empty + s, ph ^ 1, abort_sh, 40)) break;
         mbar_arrive_expect_tx(bar_ld_full + s, 2 * C::TILE + 1024);
         for (int b = 0; b < C::NBOX; ++b) {
-          tma_load_3d(smem + C::OFF_Q + s * C::TILE + b * C::BOX, &tmQ, bar_ld_full + s, b * 64, i * 128, bh);
-          tma_load_3d(smem + C::OFF_DO + s * C::TILE + b * C::BOX, &tmDO, bar_ld_full + s, b * 64, i * 128, bh);
+          tma_load_3d(smem + C::OFF_Q + s * C::TILE + b * C::BOX, &tmQ, bar_ld_full + s, b * 64, i * 128, hq);
+          tma_load_3d(smem + C::OFF_DO + s * C::TILE + b * C::BOX, &tmDO, bar_ld_full + s, b * 64, i * 128, hq);
         }
-        const size_t roff = static_cast<size_t>(bh) * a.Npad + static_cast<size_t>(i) * 128;
+        const size_t roff = static_cast<size_t>(hq) * a.Npad + static_cast<size_t>(i) * 128;
         bulk_load(smem + C::OFF_LSE + s * 512, a.lse2 + roff, 512, bar_ld_full + s);
         bulk_load(smem + C::OFF_DV + s * 512, a.dvec + roff, 512, bar_ld_full + s);
       }
@@ -312,10 +318,10 @@ __global__ void __launch_bounds__(448, 1)
     const int r = threadIdx.x - 256;  // query row in tile == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
     for (int t = 0; t < steps; ++t) {
-      const int i = i0 + t;
+      const int i = step_tile(t), hq = step_head(t);
       if (!mbar_wait(bar_dq_full, t & 1, abort_sh, 46)) break;
       tc_fence_after();
-      float* dst = a.dq_acc + (static_cast<size_t>(bh) * a.Npad + static_cast<size_t>(i) * 128 + r) * D;
+      float* dst = a.dq_acc + (static_cast<size_t>(hq) * a.Npad + static_cast<size_t>(i) * 128 + r) * D;
       const bool live = i * 128 + r < N;
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
@@ -342,7 +348,7 @@ __global__ void __launch_bounds__(448, 1)
     const float c = a.scale_log2;
     bool ok = true;
     for (int t = 0; t < steps && ok; ++t) {
-      const int i = i0 + t;
+      const int i = step_tile(t);
       const int s = t & 1;
       const float* lse2 = reinterpret_cast<const float*>(smem + C::OFF_LSE + s * 512) + half * 64;
       const float* dv = reinterpret_cast<const float*>(smem + C::OFF_DV + s * 512) + half * 64;
@@ -401,7 +407,7 @@ __global__ void __launch_bounds__(448, 1)
     if (ok) {
       tc_fence_after();
       const uint32_t col = half ? C::COL_DK : C::COL_DV;
-      __nv_bfloat16* dst = (half ? a.dk : a.dv) + (static_cast<size_t>(bh) * N + key) * D;
+      __nv_bfloat16* dst = (half ? a.dk : a.dv) + (static_cast<size_t>(bh_kv) * N + key) * D;
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t v[32];
@@ -492,11 +498,14 @@ __global__ void __launch_bounds__(448, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int N = a.N;
-  const int bh = blockIdx.x % a.BH;
-  const int j = blockIdx.x / a.BH;  // key tile of 128
-  const int n_q = (N + 63) >> 6;    // query tiles of 64
+  const int bh_kv = blockIdx.x % a.BHkv;  // key/value head
+  const int j = blockIdx.x / a.BHkv;      // key tile of 128
+  const int n_q = (N + 63) >> 6;          // query tiles of 64
   const int i0 = a.causal ? 2 * j : 0;
-  const int steps = n_q - i0;
+  const int spq = n_q - i0;               // query tiles per query head
+  const int steps = spq * a.group;        // the walk covers every query head of the group
+  auto step_head = [&](int t) { return bh_kv * a.group + t / spq; };
+  auto step_tile = [&](int t) { return i0 + t % spq; };
 
   if ((smem_u32(smem) & 1023u) != 0) {
     if (threadIdx.x == 0) atomicCAS(&g_fa_status, 0, 4 /*FA_ERR_CUDA*/ | (98 << 8));
@@ -539,22 +548,22 @@ __global__ void __launch_bounds__(448, 1)
       tma_prefetch_desc(&tmDO64);
       mbar_arrive_expect_tx(bar_kv, 2 * C::KV_TILE);
       for (int b = 0; b < 2; ++b) {
-        tma_load_3d(smem + C::OFF_K + b * C::KV_BOX, &tmK, bar_kv, b * 64, j * 128, bh);
-        tma_load_3d(smem + C::OFF_V + b * C::KV_BOX, &tmV, bar_kv, b * 64, j * 128, bh);
+        tma_load_3d(smem + C::OFF_K + b * C::KV_BOX, &tmK, bar_kv, b * 64, j * 128, bh_kv);
+        tma_load_3d(smem + C::OFF_V + b * C::KV_BOX, &tmV, bar_kv, b * 64, j * 128, bh_kv);
       }
       int t = 0;
       for (; t < steps; ++t) {
-        const int i = i0 + t;
+        const int i = step_tile(t), hq = step_head(t);
         const int s = t % C::NST;
         const uint32_t ph = (t / C::NST) & 1;
         if (!mbar_wait(bar_ld_empty + s, ph ^ 1, abort_sh, 60)) break;
         mbar_arrive_expect_tx(bar_ld_full + s, 2 * C::Q_TILE + 512);
         for (int b = 0; b < 2; ++b) {
-          tma_load_3d(smem + C::OFF_Q + s * C::Q_TILE + b * C::Q_BOX, &tmQ64, bar_ld_full + s, b * 64, i * 64, bh);
+          tma_load_3d(smem + C::OFF_Q + s * C::Q_TILE + b * C::Q_BOX, &tmQ64, bar_ld_full + s, b * 64, i * 64, hq);
           tma_load_3d(smem + C::OFF_DO + s * C::Q_TILE + b * C::Q_BOX, &tmDO64, bar_ld_full + s, b * 64, i * 64,
-                      bh);
+                      hq);
         }
-        const size_t roff = static_cast<size_t>(bh) * a.Npad + static_cast<size_t>(i) * 64;
+        const size_t roff = static_cast<size_t>(hq) * a.Npad + static_cast<size_t>(i) * 64;
         bulk_load(smem + C::OFF_LSE + s * 256, a.lse2 + roff, 256, bar_ld_full + s);
         bulk_load(smem + C::OFF_DV + s * 256, a.dvec + roff, 256, bar_ld_full + s);
       }
@@ -642,7 +651,7 @@ __global__ void __launch_bounds__(448, 1)
     const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
     for (int t = 0; t < steps; ++t) {
       const int b = t & 1;
-      const int i = i0 + t;
+      const int i = step_tile(t), hq = step_head(t);
       if (!mbar_wait(bar_dq_full + b, (t >> 1) & 1, abort_sh, 65)) break;
       tc_fence_after();
       uint32_t v[64];
@@ -651,7 +660,7 @@ __global__ void __launch_bounds__(448, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bar_dq_free + b);  // the buffer is free as soon as it is in registers
-      float* dst = a.dq_acc + (static_cast<size_t>(bh) * a.Npad + static_cast<size_t>(i) * 64) * D + c;
+      float* dst = a.dq_acc + (static_cast<size_t>(hq) * a.Npad + static_cast<size_t>(i) * 64) * D + c;
 #pragma unroll
       for (int q = 0; q < 64; ++q) atomicAdd(dst + static_cast<size_t>(q) * D, __uint_as_float(v[q]));
     }
@@ -664,7 +673,7 @@ __global__ void __launch_bounds__(448, 1)
     const float cl = a.scale_log2;
     bool ok = true;
     for (int t = 0; t < steps && ok; ++t) {
-      const int i = i0 + t;
+      const int i = step_tile(t);
       const int b = t & 1;
       const uint32_t ph = (t >> 1) & 1;
       const int st = t % C::NST;
@@ -732,7 +741,7 @@ __global__ void __launch_bounds__(448, 1)
     if (ok) {
       tc_fence_after();
       const uint32_t col = half ? C::COL_DK : C::COL_DV;
-      __nv_bfloat16* dst = (half ? a.dk : a.dv) + (static_cast<size_t>(bh) * N + key) * D;
+      __nv_bfloat16* dst = (half ? a.dk : a.dv) + (static_cast<size_t>(bh_kv) * N + key) * D;
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t v[32];

@@ -72,6 +72,7 @@ struct FwdArgs {
   const float* sk;  // [BH, nqb] per 128-row block of K
   const float* sv;  // [BH] per head of V
   int nqb;          // ceil(N / 128)
+  int group;        // query heads per key/value head (1 = multi-head attention)
 };
 
 template <typename T, int D, bool FP8P>
@@ -121,6 +122,10 @@ __global__ void __launch_bounds__(320, 1)
   const int r_in_group = blockIdx.x - group * kHeadGroup * a.nblk;
   const int bh = group * kHeadGroup + r_in_group % heads_in_group;
   int qblk = r_in_group / heads_in_group;
+  // grouped-query attention: query head bh reads key/value head bh / group (the
+  // query heads of one key/value head are adjacent, so they run side by side and
+  // share its tiles through L2)
+  const int bh_kv = bh / a.group;
   if (a.causal) qblk = a.nblk - 1 - qblk;
   const int m0 = qblk * 256;
   const int n_kv = (N + 127) >> 7;
@@ -179,12 +184,12 @@ __global__ void __launch_bounds__(320, 1)
         mbar_arrive_expect_tx(&bar_kf[s], C::TILE_BYTES);
         for (int b = 0; b < C::NBOX; ++b)
           tma_load_3d(smem + C::OFF_K + s * C::TILE_BYTES + b * C::BOX_BYTES, &tmK, &bar_kf[s], b * C::BOX_COLS,
-                      j * 128, bh);
+                      j * 128, bh_kv);
         if (!mbar_wait(&bar_ve[s], ph ^ 1, &abort_sh, 2)) break;
         mbar_arrive_expect_tx(&bar_vf[s], C::TILE_BYTES);
         for (int b = 0; b < C::NBOX; ++b)
           tma_load_3d(smem + C::OFF_V + s * C::TILE_BYTES + b * C::BOX_BYTES, &tmV, &bar_vf[s], b * C::BOX_COLS,
-                      j * 128, bh);
+                      j * 128, bh_kv);
       }
       // teardown: let every issued copy land before the CTA can exit
       const int first = max(0, n_steps - C::NSTAGE);
@@ -345,6 +350,7 @@ __global__ void __launch_bounds__(320, 1)
     // E4M3 operands carry block scales: the score factor of tile j is
     // scale*log2(e) * sq[query block] * sk[key block j]
     const float c_base = C::EB == 1 ? a.scale_log2 * a.sq[static_cast<size_t>(bh) * a.nqb + qt] : a.scale_log2;
+    const int bh_k = bh_kv;  // key-side scales are per key/value head
     float m_run = -INFINITY, l_run = 0.f;
     uint32_t fl_sink = 0, fl_non = 0;
     int cnt = 0;
@@ -353,7 +359,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int t = 0; t < n_steps; ++t) {
         const int j = rev ? n_steps - 1 - t : t;
         if (j >= kv_end) continue;
-        const float c = C::EB == 1 ? c_base * a.sk[static_cast<size_t>(bh) * a.nqb + j] : c_base;
+        const float c = C::EB == 1 ? c_base * a.sk[static_cast<size_t>(bh_k) * a.nqb + j] : c_base;
         if (!(ok = mbar_wait(&bar_s[i], cnt & 1, &abort_sh, 10 + i))) break;
         tc_fence_after();
         float sv[128];
@@ -502,7 +508,7 @@ __global__ void __launch_bounds__(320, 1)
       if (ok) ok = mbar_wait(&bar_o[i], 0, &abort_sh, 12 + i);
       if (ok) {
         tc_fence_after();
-        const float inv = (C::EB == 1 ? a.sv[bh] : 1.0f) / (l_run * a.p_scale);
+        const float inv = (C::EB == 1 ? a.sv[bh_kv] : 1.0f) / (l_run * a.p_scale);
         // output: fp32 for fp32 inputs, bf16 otherwise (also for E4M3 operands)
         using OutT = typename std::conditional<C::EB == 4, float, __nv_bfloat16>::type;
         OutT* orow = reinterpret_cast<OutT*>(a.o) + (static_cast<size_t>(bh) * N + row) * D;

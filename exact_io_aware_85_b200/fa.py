@@ -140,3 +140,24 @@ def fa_fwd_fp8(q8, k8, v8, sq, sk, sv, o, lse, causal: bool, scale: float, S: fl
     B, H, N, d = _dims(q8)
     _check(lib.fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq), _ptr(sk), _ptr(sv), _ptr(o), _ptr(lse), B, H, N,
                           d, int(causal), float(scale), float(S), int(kv_order), _stream(stream)), "fa_fwd_fp8")
+
+
+lib.fa_fwd_gqa.argtypes = [_vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _cf, _vp]
+lib.fa_bwd_gqa.argtypes = [_vp] * 9 + [_ci] * 6 + [_cf, _vp, _sz, _vp]
+
+
+def fa_fwd_gqa(q, k, v, o, lse, causal: bool, scale: float, stream=None) -> None:
+    """Grouped-query forward: k, v have H_kv heads, q and o have H (a multiple)."""
+    B, H, N, d = _dims(q)
+    Hkv = int(k.shape[1])
+    _check(lib.fa_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, N, d, int(causal), float(scale),
+                          _stream(stream)), "fa_fwd_gqa")
+
+
+def fa_bwd_gqa(q, k, v, o, do, lse, dq, dk, dv, causal: bool, scale: float, workspace, stream=None) -> None:
+    """Grouped-query backward; dk, dv have H_kv heads (group sums)."""
+    B, H, N, d = _dims(q)
+    Hkv = int(k.shape[1])
+    _check(lib.fa_bwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), B,
+                          H, Hkv, N, d, int(causal), float(scale), _ptr(workspace), int(workspace.numel()),
+                          _stream(stream)), "fa_bwd_gqa")

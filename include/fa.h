@@ -112,6 +112,23 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
 int fa_fwd_fp8p(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
                 int causal, float scale, float S, int kv_order, unsigned long long* stats, int n_sink, void* stream);
 
+/* Grouped-query / multi-query attention ("FlashAttention for Scalable Vector
+ * Architectures", "Metodologia": a key/value head shared by several query heads;
+ * "FlashAttention (IT)", "FlashAttention-2": Multi-Query Attention).
+ * q, o: [B,H,N,d]; k, v: [B,H_kv,N,d] with H a multiple of H_kv; query head h
+ * uses key/value head h / (H / H_kv).  H_kv = 1 is multi-query attention,
+ * H_kv = H is fa_fwd.  lse: [B,H,N].  Other conventions as fa_fwd. */
+int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv, int N, int d,
+               int causal, float scale, void* stream);
+
+/* Backward of fa_fwd_gqa: dq [B,H,N,d]; dk, dv [B,H_kv,N,d] are the sums of the
+ * gradients over the query heads of each group (accumulated inside the kernel,
+ * no extra pass).  workspace: fa_bwd_workspace_bytes(B, H, N, d).  Other
+ * conventions as fa_bwd. */
+int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse, void* dq,
+               void* dk, void* dv, int B, int H, int H_kv, int N, int d, int causal, float scale, void* workspace,
+               size_t workspace_bytes, void* stream);
+
 /* FP8 operands for fa_fwd_fp8 ("flash-attention-trading-models", section "FA3",
  * item 3: FP8 with incoherent processing).  Quantises bf16 q, k, v [B,H,N,d]
  * to E4M3 codes (round to nearest even, saturating):
