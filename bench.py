@@ -219,7 +219,8 @@ def config_of(w, ws):
             "FP8 P-cast forward, S=256, forward key order, sink Delta=8" if w.sink else
             "E4M3 forward (Hadamard-rotated block-quantised Q/K, per-head V, P-cast S=256)" if w.dtype == "fp8"
             else "forward (O + LSE)")
-    return {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} {w.dtype} "
+    hk = f" H_kv={w.hkv}" if w.hkv else ""
+    return {"workload": f"{w.name}: B={w.B} H={w.H}{hk} N={w.N} d={w.d} {w.dtype} "
                         f"{'causal' if w.causal else 'non-causal'} {what}",
             "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal, "parallelism": f"replicas x{ws}",
             "l2": "inputs larger than L2 (no flush needed)" if 3 * w.B * w.H * w.N * w.d * 2 > 126e6
@@ -290,6 +291,12 @@ def main():
 
         def run():
             fa.fa_fwd_fp8(q8, k8, v8, sq, sk, sv, o, lse, w.causal, w.scale, 256.0, 0)
+    elif w.hkv:
+        k = k[:, : w.hkv].contiguous()
+        v = v[:, : w.hkv].contiguous()
+
+        def run():
+            fa.fa_fwd_gqa(q, k, v, o, lse, w.causal, w.scale)
     elif w.dtype == "bf16":
         def run():
             fa.fa_fwd(q, k, v, o, lse, w.causal, w.scale)
@@ -367,7 +374,7 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, ws)
-    h2d = 3 * q.numel() * q.element_size()
+    h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
     d2h = (3 * q.numel() * q.element_size() if w.backward else o.numel() * o.element_size()) + lse.numel() * 4
     if w.backward:
         h2d += do.numel() * do.element_size()
@@ -384,6 +391,8 @@ def main():
         kernel_name = "fa_fwd_kernel<bf16,%d,FP8P>" % w.d
     elif w.dtype == "fp8":
         kernel_name = "fa_fwd_kernel<e4m3,%d> (kind::f8f6f4)" % w.d
+    elif w.hkv:
+        kernel_name = "fa_fwd_kernel<bf16,%d> grouped-query (%d query heads per key/value head)" % (w.d, w.H // w.hkv)
     else:
         kernel_name = "fa_fwd_kernel<%s,%d>" % ("bf16" if w.dtype == "bf16" else "f32/tf32", w.d)
     achieved = flops / (step_ms_local * 1e-3) / 1e12

@@ -34,6 +34,7 @@ class Workload:
     causal: bool
     backward: bool = False
     sink: bool = False
+    hkv: int = 0  # key/value heads for grouped-query attention (0: same as H)
 
     @property
     def scale(self) -> float:
@@ -57,6 +58,8 @@ WORKLOADS = {
     "sink": Workload("sink", 1, 32, 16384, 128, "bf16", False, sink=True),
     # the prefill shape on E4M3 operands (full FP8 forward with incoherent processing)
     "prefill_fp8": Workload("prefill_fp8", 4, 32, 8192, 128, "fp8", True),
+    # the prefill shape with 8 key/value heads shared by groups of 4 query heads
+    "prefill_gqa": Workload("prefill_gqa", 4, 32, 8192, 128, "bf16", True, hkv=8),
 }
 
 SINK_DELTAS = (0.0, 2.0, 4.0, 6.0, 7.0, 8.0, 10.0, 12.0)
