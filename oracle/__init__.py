@@ -17,6 +17,8 @@ Functions and the passages they follow:
   backward recomputes the scores, "Pase hacia atras"; the calculus is standard).
 * ``attn_fwd_gqa`` / ``attn_bwd_gqa`` -- grouped-query / multi-query attention as
   attention over key/value heads repeated across each query-head group.
+* ``attn_decode`` -- one decoding step: a single new query row per head against
+  the whole key/value cache (the last row of causal attention).
 * ``attn_fwd_fp8p`` -- tile-by-tile emulation of the E4M3 P-cast with static
   scale S and forward/reverse key-tile order ("P-Cast precision in FP8
   attention", sections 1-2).
@@ -69,6 +71,7 @@ def _load():
         lib.oracle_attn_fwd_fp8p.argtypes = [dp, dp, dp, dp, dp, ci, ci, ci, ci, ci, cd, cd, ci, ci, ci, ip]
         lib.oracle_fp8_quantize.argtypes = [dp, dp, dp, dp, ci, ci, ci, ci]
         lib.oracle_hadamard_rotate.argtypes = [dp, dp, dp, ctypes.c_int64, ci]
+        lib.oracle_attn_decode.argtypes = [dp, dp, dp, dp, dp, ci, ci, ci, ci, ci, cd]
         lib.oracle_num_threads.restype = ci
         _lib = lib
     return _lib
@@ -139,6 +142,18 @@ def attn_bwd_gqa(q, k, v, do, causal: bool, scale: float):
     g = Hq // Hkv
     dq, dk, dv = attn_bwd(q, np.repeat(_f64(k), g, axis=1), np.repeat(_f64(v), g, axis=1), do, causal, scale)
     return dq, dk.reshape(B, Hkv, g, N, d).sum(axis=2), dv.reshape(B, Hkv, g, N, d).sum(axis=2)
+
+
+def attn_decode(q, k, v, scale: float):
+    """One decoding step: q [B,Hq,d] (one new query row per head) against all
+    Nk cached keys of k, v [B,Hkv,Nk,d]; returns o [B,Hq,d], lse [B,Hq]."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    o = np.empty_like(q)
+    lse = np.empty((B, Hq), dtype=np.float64)
+    _load().oracle_attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nk, d, float(scale))
+    return o, lse
 
 
 def attn_fwd_fp8p(q, k, v, causal: bool, scale: float, S: float, kv_order: int, Bc: int = 128, n_sink: int = 4):

@@ -127,6 +127,26 @@ void oracle_attn_fwd_rows(const double* Q, const double* K, const double* V, con
   }
 }
 
+/* Decode step: one query row per query head against all Nk keys of its
+ * key/value head (head h uses key/value head h / (Hq / Hkv)).  Q, O [B*Hq, d];
+ * K, V [B*Hkv, Nk, d]; LSE [B*Hq]. */
+void oracle_attn_decode(const double* Q, const double* K, const double* V, double* O, double* LSE, int B, int Hq,
+                        int Hkv, int Nk, int d, double scale) {
+  const int g = Hq / Hkv;
+#pragma omp parallel
+  {
+    double* s = (double*)malloc(sizeof(double) * (size_t)(Nk > 0 ? Nk : 1));
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t t = 0; t < (int64_t)B * Hq; ++t) {
+      const int64_t b = t / Hq, h = t % Hq;
+      const int64_t kv = b * Hkv + h / g;
+      fwd_row(Q + t * d, K + kv * (int64_t)Nk * d, V + kv * (int64_t)Nk * d, Nk, d, Nk, scale, s, O + t * d,
+              LSE + t);
+    }
+    free(s);
+  }
+}
+
 /* ------------------------------------------------------------------------- */
 /* Backward: derivatives of the definition, one query row at a time           */
 /* ------------------------------------------------------------------------- */
