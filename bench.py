@@ -291,6 +291,18 @@ def main():
 
         def run():
             fa.fa_fwd_fp8(q8, k8, v8, sq, sk, sv, o, lse, w.causal, w.scale, 256.0, 0)
+    elif w.decode:
+        # q, o: one row per head; k, v: the cache of H_kv heads
+        q = q[:, :, 0].contiguous()
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.H), dtype=torch.float32, device="cuda")
+        k = k[:, : w.hkv].contiguous()
+        v = v[:, : w.hkv].contiguous()
+        ws_dec = torch.empty(fa.fa_decode_workspace_bytes(w.B, w.H, w.hkv, w.N, w.d), dtype=torch.uint8,
+                             device="cuda")
+
+        def run():
+            fa.fa_decode(q, k, v, o, lse, w.scale, ws_dec)
     elif w.hkv:
         k = k[:, : w.hkv].contiguous()
         v = v[:, : w.hkv].contiguous()
@@ -385,17 +397,28 @@ def main():
         # no measured FP8 peak on this machine: the measured bf16 peak x the nominal 2x FP8 ratio
         peak *= 2.0
         peak_note = f"{peak_src} bf16 burst x 2 (nominal FP8/BF16 ratio)"
+    bound, unit, peak_val = "tensor", "TFLOP/s", peak
+    if w.decode:
+        # bound by reading the key/value cache: roofline in bytes against measured HBM
+        bound, unit = "hbm", "GB/s"
+        peak_val = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        peak_note = f"{peak_src} HBM copy bandwidth (MEASURED_PEAKS.json)"
     if w.backward:
         kernel_name = "training step: fa_fwd_kernel<bf16,%d> + fa_bwd (pre, main, post)" % w.d
     elif w.sink:
         kernel_name = "fa_fwd_kernel<bf16,%d,FP8P>" % w.d
     elif w.dtype == "fp8":
         kernel_name = "fa_fwd_kernel<e4m3,%d> (kind::f8f6f4)" % w.d
+    elif w.decode:
+        kernel_name = "fa_decode_split_kernel<%d> + fa_decode_combine_kernel<%d>" % (w.d, w.d)
     elif w.hkv:
         kernel_name = "fa_fwd_kernel<bf16,%d> grouped-query (%d query heads per key/value head)" % (w.d, w.H // w.hkv)
     else:
         kernel_name = "fa_fwd_kernel<%s,%d>" % ("bf16" if w.dtype == "bf16" else "f32/tf32", w.d)
     achieved = flops / (step_ms_local * 1e-3) / 1e12
+    if w.decode:
+        achieved_bytes = (sum(t.numel() * t.element_size() for t in (q, k, v, o)) + lse.numel() * 4) / (
+            step_ms_local * 1e-3) / 1e9
     tr = TRAFFIC.get(w.name, {})
     traffic = tr.get("bytes") if tr.get("fwd_src_sha1") == _src_hash() else None
     clocks = clk.summary()
@@ -410,8 +433,9 @@ def main():
             "pct_of_peak": {"measured_bf16_burst": achieved / peak,
                             "measured_bf16_sustained": achieved / float(peaks.get("bf16_tflops_sustained", 1390.0)),
                             "datasheet_bf16_2250": achieved / 2250.0},
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "peak_source": peak_note,
+            "roofline": {"bound": bound, "achieved": achieved_bytes if w.decode else achieved,
+                         "peak": peak_val, "unit": unit,
+                         "frac": (achieved_bytes if w.decode else achieved) / peak_val, "peak_source": peak_note,
                          "traffic": traffic, "kernel": kernel_name,
                          "launch_ms": {"median": statistics.median(launch_ms), "min": min(launch_ms),
                                        "mean": step_ms_local}},

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -16,6 +17,7 @@
 #include "fwd.cuh"
 #include "bwd.cuh"
 #include "fp8.cuh"
+#include "decode.cuh"
 
 namespace fa {
 // Self-test of the failure path: waits on an mbarrier that nothing will ever
@@ -239,6 +241,19 @@ int noalloc_scratch_for_current_device(void** out) {
   *out = g_noalloc_ptr[dev];
   return FA_OK;
 }
+// Decode split plan: enough key chunks that B * H_kv * chunks is about sixteen
+// CTAs per SM (148 SMs; two are resident at a time), so the last wave is a small
+// fraction of the work; chunks of whole 64-key tiles.  A pure function of the
+// sizes, so the workspace size is known before any launch.
+void decode_plan(int B, int Hkv, int N, int* nsplit, int* tiles_per_split) {
+  const int tiles = (N + fa::kDecKT - 1) / fa::kDecKT;
+  const int bhkv = B * Hkv;
+  const int target = std::max(1, (16 * 148 + bhkv - 1) / bhkv);
+  const int ns = std::min(tiles, target);
+  *tiles_per_split = (tiles + ns - 1) / ns;
+  *nsplit = (tiles + *tiles_per_split - 1) / *tiles_per_split;
+}
+
 }  // namespace
 
 extern "C" {
@@ -302,6 +317,61 @@ int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return d == 64 ? launch_bwd<64>(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, causal, scale, workspace, s, H_kv)
                  : launch_bwd<128>(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, causal, scale, workspace, s, H_kv);
+}
+
+size_t fa_decode_workspace_bytes(int B, int H, int H_kv, int N, int d) {
+  if (B < 1 || H < 1 || H_kv < 1 || N < 1 || H % H_kv != 0 || (d != 64 && d != 128)) return 0;
+  int ns, tps;
+  decode_plan(B, H_kv, N, &ns, &tps);
+  const size_t bytes = static_cast<size_t>(ns) * B * H * (static_cast<size_t>(d) + 2) * sizeof(float);
+  return (bytes + 255) / 256 * 256;
+}
+
+int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv, int N, int d,
+              float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !lse || !workspace) return FA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || H_kv < 1 || N < 1 || H % H_kv != 0) return FA_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const int g = H / H_kv;
+  if (g > fa::kDecMaxG) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H_kv * N * d >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 15u))
+    return FA_ERR_ALIGNMENT;
+  if (workspace_bytes < fa_decode_workspace_bytes(B, H, H_kv, N, d)) return FA_ERR_INVALID_ARG;
+  fa::DecodeArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.v = static_cast<const __nv_bfloat16*>(v);
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.N = N;
+  a.BHkv = B * H_kv;
+  a.g = g;
+  decode_plan(B, H_kv, N, &a.nsplit, &a.tiles_per_split);
+  a.part_o = static_cast<float*>(workspace);
+  a.part_ml = a.part_o + static_cast<size_t>(a.nsplit) * B * H * d;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const dim3 grid(a.nsplit, a.BHkv);
+  cudaError_t e;
+  if (d == 64) {
+    constexpr int SM = sizeof(fa::DecodeSmem<64>);
+    e = cudaFuncSetAttribute(fa::fa_decode_split_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, SM);
+    if (e != cudaSuccess) return cuda_fail(e);
+    fa::fa_decode_split_kernel<64><<<grid, fa::kDecThreads, SM, s>>>(a);
+    fa::fa_decode_combine_kernel<64><<<B * H, 64, 0, s>>>(a);
+  } else {
+    constexpr int SM = sizeof(fa::DecodeSmem<128>);
+    e = cudaFuncSetAttribute(fa::fa_decode_split_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, SM);
+    if (e != cudaSuccess) return cuda_fail(e);
+    fa::fa_decode_split_kernel<128><<<grid, fa::kDecThreads, SM, s>>>(a);
+    fa::fa_decode_combine_kernel<128><<<B * H, 128, 0, s>>>(a);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return FA_OK;
 }
 
 int fa_fp8_quantize(const void* q, const void* k, const void* v, const float* signs, void* q8, void* k8, void* v8,

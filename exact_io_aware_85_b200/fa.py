@@ -161,3 +161,20 @@ def fa_bwd_gqa(q, k, v, o, do, lse, dq, dk, dv, causal: bool, scale: float, work
     _check(lib.fa_bwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), B,
                           H, Hkv, N, d, int(causal), float(scale), _ptr(workspace), int(workspace.numel()),
                           _stream(stream)), "fa_bwd_gqa")
+
+
+lib.fa_decode_workspace_bytes.restype = _sz
+lib.fa_decode_workspace_bytes.argtypes = [_ci] * 5
+lib.fa_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _cf, _vp, _sz, _vp]
+
+
+def fa_decode_workspace_bytes(B: int, H: int, H_kv: int, N: int, d: int) -> int:
+    return int(lib.fa_decode_workspace_bytes(B, H, H_kv, N, d))
+
+
+def fa_decode(q, k, v, o, lse, scale: float, workspace, stream=None) -> None:
+    """One decoding step: q, o [B,H,d]; k, v [B,H_kv,N,d]; lse [B,H]."""
+    B, H, d = (int(x) for x in q.shape)
+    Hkv, N = int(k.shape[1]), int(k.shape[2])
+    _check(lib.fa_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, N, d, float(scale),
+                         _ptr(workspace), int(workspace.numel()), _stream(stream)), "fa_decode")

@@ -35,13 +35,17 @@ class Workload:
     backward: bool = False
     sink: bool = False
     hkv: int = 0  # key/value heads for grouped-query attention (0: same as H)
+    decode: bool = False  # one query row per head against an N-key cache
 
     @property
     def scale(self) -> float:
         return 1.0 / math.sqrt(self.d)
 
     def fwd_flops(self) -> float:
-        """4 B H N^2 d for the two matmuls, halved when causal (N^2/2 convention)."""
+        """4 B H N^2 d for the two matmuls, halved when causal (N^2/2 convention);
+        4 B H N d for a decoding step (one query row per head)."""
+        if self.decode:
+            return 4.0 * self.B * self.H * self.N * self.d
         f = 4.0 * self.B * self.H * self.N * self.N * self.d
         return f / 2.0 if self.causal else f
 
@@ -60,6 +64,8 @@ WORKLOADS = {
     "prefill_fp8": Workload("prefill_fp8", 4, 32, 8192, 128, "fp8", True),
     # the prefill shape with 8 key/value heads shared by groups of 4 query heads
     "prefill_gqa": Workload("prefill_gqa", 4, 32, 8192, 128, "bf16", True, hkv=8),
+    # one decoding step of 8 sequences against a 32K-token key/value cache, 8 KV heads
+    "decode": Workload("decode", 8, 32, 32768, 128, "bf16", False, hkv=8, decode=True),
 }
 
 SINK_DELTAS = (0.0, 2.0, 4.0, 6.0, 7.0, 8.0, 10.0, 12.0)

@@ -129,6 +129,18 @@ int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const
                void* dk, void* dv, int B, int H, int H_kv, int N, int d, int causal, float scale, void* workspace,
                size_t workspace_bytes, void* stream);
 
+/* One decoding step: for each query head a single new query row attends to all
+ * N cached keys of its key/value head (the last row of causal attention,
+ * "flash-attention-trading-models", "El algoritmo de atencion flash").  Bound by
+ * reading the cache, so it runs on the CUDA cores, split over the key sequence
+ * with a log-sum-exp merge of the chunks; the g = H / H_kv query heads of a
+ * key/value head are served from one read of it (g <= 16).
+ * q, o: bf16 [B,H,d]; k, v: bf16 [B,H_kv,N,d]; lse: fp32 [B,H].
+ * workspace: caller-owned, >= fa_decode_workspace_bytes(), 16-byte aligned. */
+size_t fa_decode_workspace_bytes(int B, int H, int H_kv, int N, int d);
+int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv, int N, int d,
+              float scale, void* workspace, size_t workspace_bytes, void* stream);
+
 /* FP8 operands for fa_fwd_fp8 ("flash-attention-trading-models", section "FA3",
  * item 3: FP8 with incoherent processing).  Quantises bf16 q, k, v [B,H,N,d]
  * to E4M3 codes (round to nearest even, saturating):
