@@ -413,6 +413,8 @@ def main():
         kernel_name = "fa_decode_split_kernel<%d> + fa_decode_combine_kernel<%d>" % (w.d, w.d)
     elif w.hkv:
         kernel_name = "fa_fwd_kernel<bf16,%d> grouped-query (%d query heads per key/value head)" % (w.d, w.H // w.hkv)
+    elif w.d == 256:
+        kernel_name = "fa_fwd256_kernel (one Q tile per CTA, double-buffered S)"
     else:
         kernel_name = "fa_fwd_kernel<%s,%d>" % ("bf16" if w.dtype == "bf16" else "f32/tf32", w.d)
     achieved = flops / (step_ms_local * 1e-3) / 1e12

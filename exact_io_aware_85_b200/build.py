@@ -7,7 +7,7 @@ import subprocess
 PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libfa.so")
-SOURCES = ["api.cu", "sm100.cuh", "fwd.cuh", "bwd.cuh", "fp8.cuh", "decode.cuh"]
+SOURCES = ["api.cu", "sm100.cuh", "fwd.cuh", "bwd.cuh", "fp8.cuh", "decode.cuh", "fwd256.cuh"]
 HEADER = os.path.join(os.path.dirname(PKG), "include", "fa.h")
 
 

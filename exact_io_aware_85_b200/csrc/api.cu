@@ -18,6 +18,7 @@
 #include "bwd.cuh"
 #include "fp8.cuh"
 #include "decode.cuh"
+#include "fwd256.cuh"
 
 namespace fa {
 // Self-test of the failure path: waits on an mbarrier that nothing will ever
@@ -81,11 +82,11 @@ int encode_qkv_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int
 }
 
 int check_common(const void* q, const void* k, const void* v, const void* o, const void* lse, int B, int H, int N,
-                 int d, float scale) {
+                 int d, float scale, bool allow256 = false) {
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
   if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && !(allow256 && d == 256)) return FA_ERR_UNSUPPORTED;
   const long long total = static_cast<long long>(B) * H * N * d;
   if (total >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGNMENT;
@@ -241,6 +242,35 @@ int noalloc_scratch_for_current_device(void** out) {
   *out = g_noalloc_ptr[dev];
   return FA_OK;
 }
+// Head dim 256: one 128-row Q tile per CTA, 64-key K/V tiles (fwd256.cuh).
+int launch_fwd256(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv, int N,
+                  int causal, float scale, cudaStream_t stream) {
+  using C = fa::Fwd256Cfg;
+  const auto dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUtensorMap mq, mk, mv;
+  int st;
+  if ((st = encode_qkv_map(&mq, q, dt, 2, 256, N, B * H, CU_TENSOR_MAP_SWIZZLE_128B, 128)) != FA_OK) return st;
+  if ((st = encode_qkv_map(&mk, k, dt, 2, 256, N, B * Hkv, CU_TENSOR_MAP_SWIZZLE_128B, 64)) != FA_OK) return st;
+  if ((st = encode_qkv_map(&mv, v, dt, 2, 256, N, B * Hkv, CU_TENSOR_MAP_SWIZZLE_128B, 64)) != FA_OK) return st;
+  fa::Fwd256Args a;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.N = N;
+  a.BH = B * H;
+  a.nblk = (N + 127) / 128;
+  a.group = H / Hkv;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.causal = causal ? 1 : 0;
+  cudaError_t e = cudaFuncSetAttribute(fa::fa_fwd256_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::SMEM_BYTES);
+  if (e != cudaSuccess) return cuda_fail(e);
+  fa::fa_fwd256_kernel<<<static_cast<unsigned>(static_cast<long long>(a.nblk) * a.BH), C::NTHREADS, C::SMEM_BYTES,
+                         stream>>>(mq, mk, mv, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return FA_OK;
+}
+
 // Decode split plan: enough key chunks that B * H_kv * chunks is about sixteen
 // CTAs per SM (148 SMs; two are resident at a time), so the last wave is a small
 // fraction of the work; chunks of whole 64-key tiles.  A pure function of the
@@ -260,9 +290,10 @@ extern "C" {
 
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d, int causal,
            float scale, void* stream) {
-  int st = check_common(q, k, v, o, lse, B, H, N, d, scale);
+  int st = check_common(q, k, v, o, lse, B, H, N, d, scale, true);
   if (st != FA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 256) return launch_fwd256(q, k, v, o, lse, B, H, H, N, causal, scale, s);
   if (d == 64) return launch_fwd<__nv_bfloat16, 64, false>(q, k, v, o, lse, B, H, N, causal, scale, 1.f, 0, nullptr, 0, s);
   return launch_fwd<__nv_bfloat16, 128, false>(q, k, v, o, lse, B, H, N, causal, scale, 1.f, 0, nullptr, 0, s);
 }
@@ -293,10 +324,11 @@ int fa_fwd_fp8p(const void* q, const void* k, const void* v, void* o, float* lse
 
 int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv, int N, int d,
                int causal, float scale, void* stream) {
-  int st = check_common(q, k, v, o, lse, B, H, N, d, scale);
+  int st = check_common(q, k, v, o, lse, B, H, N, d, scale, true);
   if (st != FA_OK) return st;
   if (H_kv < 1 || H % H_kv != 0) return FA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 256) return launch_fwd256(q, k, v, o, lse, B, H, H_kv, N, causal, scale, s);
   if (d == 64)
     return launch_fwd<__nv_bfloat16, 64, false>(q, k, v, o, lse, B, H, N, causal, scale, 1.f, 0, nullptr, 0, s,
                                                 nullptr, nullptr, nullptr, H_kv);

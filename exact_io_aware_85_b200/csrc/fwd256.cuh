@@ -1,0 +1,278 @@
+// fwd256.cuh — exact attention forward for head dim 256 ("FlashAttention (IT)",
+// "FlashAttention-2": head dimension up to 256), same algorithm as fwd.cuh.
+//
+// At d = 256 the fp32 output tile of 128 query rows alone takes 256 of the 512
+// tensor-memory columns, so the two-Q-tile ping-pong of fwd.cuh does not fit.
+// Here a CTA owns one 128-row Q tile and walks 64-key K/V tiles; the score tile
+// is double-buffered instead, so the tensor core computes S(j+1) = Q K_{j+1}^T
+// while the softmax warps work on S(j):
+//   TMEM: S buffers [0,64) and [64,128) (P written over them as bf16), O [256,512)
+//   SMEM: Q 64 KB (resident), K and V rings of 2 x 32 KB
+// MMA order: S(0), S(1), PV(0), S(2), PV(1), S(3), ...  S(j+2) reuses the
+// buffer of S(j) and is issued after PV(j) (tcgen05 MMAs of one thread execute
+// in order).  Because S(j+1) is issued before PV(j), "S(j+1) ready" does not
+// imply "PV(j) done": a softmax thread that must rescale O (the lazy correction
+// fires only when the row max grows by more than 2^8) first waits for PV(j).
+#pragma once
+#include "sm100.cuh"
+
+namespace fa {
+
+struct Fwd256Args {
+  __nv_bfloat16* o;
+  float* lse;
+  int N, BH, nblk, group;
+  float scale_log2;
+  int causal;
+};
+
+struct Fwd256Cfg {
+  static constexpr int D = 256;
+  static constexpr int BM = 128, BN = 64;
+  static constexpr int Q_BOX = 128 * 128;   // 128 rows x 128 B (64 columns)
+  static constexpr int KV_BOX = 64 * 128;   // 64 rows x 128 B
+  static constexpr int Q_BYTES = 4 * Q_BOX;     // 64 KB
+  static constexpr int KV_BYTES = 4 * KV_BOX;   // 32 KB
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;   // 2 stages
+  static constexpr int OFF_V = OFF_K + 2 * KV_BYTES;
+  static constexpr int SMEM_BYTES = OFF_V + 2 * KV_BYTES + 1024;
+  static constexpr uint32_t COL_S = 0, COL_O = 256;  // S buffers at 0 and 64
+  static constexpr int NTHREADS = 192;
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+};
+
+__global__ void __launch_bounds__(192, 1)
+    fa_fwd256_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const Fwd256Args a) {
+  using C = Fwd256Cfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ uint64_t bar_q, bar_kf[2], bar_ke[2], bar_vf[2], bar_ve[2], bar_s[2], bar_p[2], bar_pv, bar_o, bar_done;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- work decode: query blocks of 8 adjacent heads together, heaviest first ----
+  constexpr int kHeadGroup = 8;
+  const int N = a.N;
+  const int grp = blockIdx.x / (kHeadGroup * a.nblk);
+  const int heads_in_group = min(kHeadGroup, a.BH - grp * kHeadGroup);
+  const int r_in = blockIdx.x - grp * kHeadGroup * a.nblk;
+  const int bh = grp * kHeadGroup + r_in % heads_in_group;
+  int qt = r_in / heads_in_group;
+  if (a.causal) qt = a.nblk - 1 - qt;
+  const int m0 = qt * 128;
+  const int bh_kv = bh / a.group;
+  const int n_kv = (N + 63) >> 6;
+  const int T = a.causal ? min(n_kv, 2 * qt + 2) : n_kv;  // key tiles this Q tile sees
+
+  if (warp == 5) {
+    tmem_alloc(&tmem_base_sh, 512);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    abort_sh = 0;
+    mbar_init(&bar_q, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar_kf[s], 1);
+      mbar_init(&bar_ke[s], 1);
+      mbar_init(&bar_vf[s], 1);
+      mbar_init(&bar_ve[s], 1);
+      mbar_init(&bar_s[s], 1);
+      mbar_init(&bar_p[s], 128);
+    }
+    mbar_init(&bar_pv, 1);
+    mbar_init(&bar_o, 1);
+    mbar_init(&bar_done, 1);
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp == 4) {
+    // ============================ producer ===================================
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      mbar_arrive_expect_tx(&bar_q, C::Q_BYTES);
+      for (int b = 0; b < 4; ++b) tma_load_3d(smem + C::OFF_Q + b * C::Q_BOX, &tmQ, &bar_q, b * 64, m0, bh);
+      int t = 0;
+      for (; t < T; ++t) {
+        const int s = t & 1;
+        const uint32_t ph = (t >> 1) & 1;
+        if (!mbar_wait(&bar_ke[s], ph ^ 1, &abort_sh, 80)) break;
+        mbar_arrive_expect_tx(&bar_kf[s], C::KV_BYTES);
+        for (int b = 0; b < 4; ++b)
+          tma_load_3d(smem + C::OFF_K + s * C::KV_BYTES + b * C::KV_BOX, &tmK, &bar_kf[s], b * 64, t * 64, bh_kv);
+        if (!mbar_wait(&bar_ve[s], ph ^ 1, &abort_sh, 81)) break;
+        mbar_arrive_expect_tx(&bar_vf[s], C::KV_BYTES);
+        for (int b = 0; b < 4; ++b)
+          tma_load_3d(smem + C::OFF_V + s * C::KV_BYTES + b * C::KV_BOX, &tmV, &bar_vf[s], b * 64, t * 64, bh_kv);
+      }
+      mbar_wait_drain(&bar_q, 0, 100000000ull);
+      for (int u = max(0, t - 2); u < t; ++u) {
+        mbar_wait_drain(&bar_kf[u & 1], (u >> 1) & 1, 100000000ull);
+        mbar_wait_drain(&bar_vf[u & 1], (u >> 1) & 1, 100000000ull);
+      }
+    }
+  } else if (warp == 5) {
+    // ============================ MMA issuer =================================
+    if (lane == 0) {
+      constexpr uint32_t id_s = make_idesc(128, 64, kFmtBF16, 0, 0);   // S = Q K^T: N = 64 keys, K = 256
+      constexpr uint32_t id_pv = make_idesc(128, 256, kFmtBF16, 0, 1); // O += P V: N = 256, K = 64 keys
+      const uint32_t q_addr = smem_u32(smem + C::OFF_Q);
+      const uint32_t k_addr = smem_u32(smem + C::OFF_K), v_addr = smem_u32(smem + C::OFF_V);
+      auto issue_s = [&](int t) {
+        const int s = t & 1;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const uint32_t qa = q_addr + (k >> 2) * C::Q_BOX + (k & 3) * 32;
+          const uint32_t ka = k_addr + s * C::KV_BYTES + (k >> 2) * C::KV_BOX + (k & 3) * 32;
+          mma_ss(tmem + C::COL_S + 64 * s, make_sdesc_sw128(qa, 16, 1024), make_sdesc_sw128(ka, 16, 1024), id_s,
+                 k > 0);
+        }
+        mma_commit(&bar_s[s]);
+        mma_commit(&bar_ke[s]);
+      };
+      bool ok = mbar_wait(&bar_q, 0, &abort_sh, 82);
+      for (int t = 0; ok && t < min(T, 2); ++t) {
+        if (!(ok = mbar_wait(&bar_kf[t & 1], 0, &abort_sh, 83))) break;
+        tc_fence_after();
+        issue_s(t);
+      }
+      for (int t = 0; ok && t < T; ++t) {
+        const int s = t & 1;
+        const uint32_t ph = (t >> 1) & 1;
+        if (!(ok = mbar_wait(&bar_vf[s], ph, &abort_sh, 84))) break;
+        if (!(ok = mbar_wait(&bar_p[s], ph, &abort_sh, 85))) break;
+        tc_fence_after();
+        // O += P(t) V(t): A = P from TMEM (bf16, 16 keys = 8 columns per step), B = V MN-major
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          mma_ts(tmem + C::COL_O, tmem + C::COL_S + 64 * s + k * 8,
+                 make_sdesc_sw128(v_addr + s * C::KV_BYTES + k * 2048, C::KV_BOX, 1024), id_pv,
+                 (t > 0 || k > 0) ? 1u : 0u);
+        mma_commit(&bar_ve[s]);
+        mma_commit(&bar_pv);
+        if (t + 2 < T) {
+          if (!(ok = mbar_wait(&bar_kf[s], ph ^ 1, &abort_sh, 86))) break;
+          tc_fence_after();
+          issue_s(t + 2);
+        }
+      }
+      if (ok) mma_commit(&bar_o);
+      mma_commit(&bar_done);
+      mbar_wait_drain(&bar_done, 0, 100000000ull);
+    }
+  } else {
+    // ============================ softmax warps ==============================
+    const int r = threadIdx.x;  // row in tile == TMEM lane
+    const int row = m0 + r;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;
+    const float c = a.scale_log2;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int t = 0; t < T && ok; ++t) {
+      const int s = t & 1;
+      if (!(ok = mbar_wait(&bar_s[s], (t >> 1) & 1, &abort_sh, 87))) break;
+      tc_fence_after();
+      float sv[64];
+      const uint32_t tS = tmem + lane_base + C::COL_S + 64 * s;
+      tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      tmem_wait_ld();
+      const int kbase = t * 64;
+      if (kbase + 64 > N || (a.causal && kbase + 63 > m0)) {
+        const int lim = a.causal ? min(N - 1, row) : N - 1;
+#pragma unroll
+        for (int e = 0; e < 64; ++e)
+          if (kbase + e > lim) sv[e] = -INFINITY;
+      }
+      float mx8[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) mx8[u] = fmax3(sv[u], sv[u + 8], sv[u + 16]);
+#pragma unroll
+      for (int e = 24; e < 64; e += 8)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mx8[u] = fmaxf(mx8[u], sv[e + u]);
+      const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+      float m_new = fmaxf(m_run, mx * c);
+      if (m_new - m_run <= 8.0f) m_new = m_run;  // lazy correction (exps stay <= 2^8)
+      const float alpha = ex2_approx(m_run - m_new);
+      const bool rescale = t > 0 && __any_sync(0xffffffffu, m_new != m_run);
+      l_run *= alpha;
+      m_run = m_new;
+      const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_run, -m_run);
+      float2 rs4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      uint32_t pk[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float2 x = ffma2(make_float2(sv[2 * e], sv[2 * e + 1]), c2, nm2);
+        const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
+        rs4[e & 3] = fadd2(rs4[e & 3], make_float2(p0, p1));
+        pk[e] = pack_bf16x2(p0, p1);
+      }
+      tmem_st32(tS, pk);
+      if (rescale) {
+        // PV(t-1) may still be accumulating into O: wait for it before touching O
+        if (!(ok = mbar_wait(&bar_pv, (t - 1) & 1, &abort_sh, 88))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          uint32_t ov[32];
+          tmem_ld32(tmem + lane_base + C::COL_O + ch * 32, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float2 r2 = fmul2(make_float2(__uint_as_float(ov[e]), __uint_as_float(ov[e + 1])),
+                                    make_float2(alpha, alpha));
+            ov[e] = __float_as_uint(r2.x);
+            ov[e + 1] = __float_as_uint(r2.y);
+          }
+          tmem_st32(tmem + lane_base + C::COL_O + ch * 32, ov);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar_p[s]);
+      const float2 t01 = fadd2(rs4[0], rs4[1]), t23 = fadd2(rs4[2], rs4[3]);
+      const float2 tt = fadd2(t01, t23);
+      l_run += tt.x + tt.y;
+    }
+    if (ok) ok = mbar_wait(&bar_o, 0, &abort_sh, 89);
+    if (ok) {
+      tc_fence_after();
+      const float inv = 1.0f / l_run;
+      __nv_bfloat16* orow = a.o + (static_cast<size_t>(bh) * N + row) * C::D;
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        uint32_t ov[32];
+        tmem_ld32(tmem + lane_base + C::COL_O + ch * 32, ov);
+        tmem_wait_ld();
+        if (row < N) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            dst[v4] = make_uint4(pack_bf16x2(__uint_as_float(ov[8 * v4 + 0]) * inv, __uint_as_float(ov[8 * v4 + 1]) * inv),
+                                 pack_bf16x2(__uint_as_float(ov[8 * v4 + 2]) * inv, __uint_as_float(ov[8 * v4 + 3]) * inv),
+                                 pack_bf16x2(__uint_as_float(ov[8 * v4 + 4]) * inv, __uint_as_float(ov[8 * v4 + 5]) * inv),
+                                 pack_bf16x2(__uint_as_float(ov[8 * v4 + 6]) * inv, __uint_as_float(ov[8 * v4 + 7]) * inv));
+        }
+      }
+      if (row < N) a.lse[static_cast<size_t>(bh) * N + row] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fa

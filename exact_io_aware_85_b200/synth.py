@@ -64,6 +64,8 @@ WORKLOADS = {
     "prefill_fp8": Workload("prefill_fp8", 4, 32, 8192, 128, "fp8", True),
     # the prefill shape with 8 key/value heads shared by groups of 4 query heads
     "prefill_gqa": Workload("prefill_gqa", 4, 32, 8192, 128, "bf16", True, hkv=8),
+    # head dim 256 at the prefill scale (the same FLOPs as the d=128 prefill)
+    "prefill_d256": Workload("prefill_d256", 4, 16, 8192, 256, "bf16", True),
     # one decoding step of 8 sequences against a 32K-token key/value cache, 8 KV heads
     "decode": Workload("decode", 8, 32, 32768, 128, "bf16", False, hkv=8, decode=True),
 }
