@@ -32,15 +32,19 @@ sys.path.insert(0, ROOT)
 from exact_io_aware_85_b200 import synth  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM traffic per launch of the forward kernel on the prefill workload, from the
-# ncu capture summarised in profiles/fa_fwd_prefill.md; only reported while the
-# kernel source still hashes to the value it was measured with.
-TRAFFIC = {"prefill": {"bytes": 808392448 + 261109760, "fwd_src_sha1": "66a02bcc9e41143f202698011413cec4ff2bf470"}}
+# DRAM traffic per launch of the dominant kernel, from the ncu captures summarised
+# in profiles/ (fa_fwd_prefill.md, fa_decode.md); reported only while the kernel
+# sources still hash to the values they were measured with.
+TRAFFIC = {
+    "prefill": {"bytes": 811046400 + 264259840, "src": ("fwd.cuh", "sm100.cuh"),
+                "sha1": "7423259134f17bc9027b22ed228273450d627ac3"},
+    "decode": {"bytes": 1082300000, "src": ("decode.cuh", "sm100.cuh"), "sha1": "952ee5a7e1f9132f76d788fe16a32974ec02b1b2"},
+}
 
 
-def _src_hash() -> str:
+def _src_hash(files) -> str:
     h = hashlib.sha1()
-    for f in ("fwd.cuh", "sm100.cuh"):
+    for f in files:
         with open(os.path.join(ROOT, "exact_io_aware_85_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
@@ -421,8 +425,8 @@ def main():
     if w.decode:
         achieved_bytes = (sum(t.numel() * t.element_size() for t in (q, k, v, o)) + lse.numel() * 4) / (
             step_ms_local * 1e-3) / 1e9
-    tr = TRAFFIC.get(w.name, {})
-    traffic = tr.get("bytes") if tr.get("fwd_src_sha1") == _src_hash() else None
+    tr = TRAFFIC.get(w.name)
+    traffic = tr["bytes"] if tr and tr["sha1"] == _src_hash(tr["src"]) else None
     clocks = clk.summary()
 
     if rank == 0:
