@@ -275,10 +275,23 @@ int launch_fwd256(const void* q, const void* k, const void* v, void* o, float* l
 // CTAs per SM (148 SMs; two are resident at a time), so the last wave is a small
 // fraction of the work; chunks of whole 64-key tiles.  A pure function of the
 // sizes, so the workspace size is known before any launch.
+template <int D, int NT>
+cudaError_t launch_decode_split(dim3 grid, cudaStream_t s, const CUtensorMap& mk, const CUtensorMap& mv,
+                                const fa::DecodeArgs& a) {
+  constexpr int smem = fa::DecodeLayout<D>::BYTES;
+  cudaError_t e = cudaFuncSetAttribute(fa::fa_decode_split_kernel<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       smem);
+  if (e != cudaSuccess) return e;
+  fa::fa_decode_split_kernel<D, NT><<<grid, fa::kDecThreads, smem, s>>>(mk, mv, a);
+  return cudaSuccess;
+}
+
+// Key chunks per key/value head: one wave of split CTAs (one per SM), so that
+// the pipeline of each CTA fills once and streams a long chunk.
 void decode_plan(int B, int Hkv, int N, int* nsplit, int* tiles_per_split) {
   const int tiles = (N + fa::kDecKT - 1) / fa::kDecKT;
   const int bhkv = B * Hkv;
-  const int target = std::max(1, (16 * 148 + bhkv - 1) / bhkv);
+  const int target = std::max(1, 148 / bhkv);
   const int ns = std::min(tiles, target);
   *tiles_per_split = (tiles + ns - 1) / ns;
   *nsplit = (tiles + *tiles_per_split - 1) / *tiles_per_split;
@@ -374,8 +387,6 @@ int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, 
   if (workspace_bytes < fa_decode_workspace_bytes(B, H, H_kv, N, d)) return FA_ERR_INVALID_ARG;
   fa::DecodeArgs a;
   a.q = static_cast<const __nv_bfloat16*>(q);
-  a.k = static_cast<const __nv_bfloat16*>(k);
-  a.v = static_cast<const __nv_bfloat16*>(v);
   a.o = static_cast<__nv_bfloat16*>(o);
   a.lse = lse;
   a.N = N;
@@ -386,19 +397,21 @@ int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, 
   a.part_ml = a.part_o + static_cast<size_t>(a.nsplit) * B * H * d;
   a.scale_log2 = scale * 1.4426950408889634f;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // K and V as [B*H_kv, N, d] in 128-key x 64-column boxes, 128-byte swizzled
+  CUtensorMap mk, mv;
+  int st;
+  const auto dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if ((st = encode_qkv_map(&mk, k, dt, 2, d, N, B * H_kv, CU_TENSOR_MAP_SWIZZLE_128B, fa::kDecKT)) != FA_OK) return st;
+  if ((st = encode_qkv_map(&mv, v, dt, 2, d, N, B * H_kv, CU_TENSOR_MAP_SWIZZLE_128B, fa::kDecKT)) != FA_OK) return st;
   const dim3 grid(a.nsplit, a.BHkv);
   cudaError_t e;
   if (d == 64) {
-    constexpr int SM = sizeof(fa::DecodeSmem<64>);
-    e = cudaFuncSetAttribute(fa::fa_decode_split_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, SM);
+    e = g <= 8 ? launch_decode_split<64, 1>(grid, s, mk, mv, a) : launch_decode_split<64, 2>(grid, s, mk, mv, a);
     if (e != cudaSuccess) return cuda_fail(e);
-    fa::fa_decode_split_kernel<64><<<grid, fa::kDecThreads, SM, s>>>(a);
     fa::fa_decode_combine_kernel<64><<<B * H, 64, 0, s>>>(a);
   } else {
-    constexpr int SM = sizeof(fa::DecodeSmem<128>);
-    e = cudaFuncSetAttribute(fa::fa_decode_split_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, SM);
+    e = g <= 8 ? launch_decode_split<128, 1>(grid, s, mk, mv, a) : launch_decode_split<128, 2>(grid, s, mk, mv, a);
     if (e != cudaSuccess) return cuda_fail(e);
-    fa::fa_decode_split_kernel<128><<<grid, fa::kDecThreads, SM, s>>>(a);
     fa::fa_decode_combine_kernel<128><<<B * H, 128, 0, s>>>(a);
   }
   e = cudaGetLastError();
