@@ -443,10 +443,13 @@ __global__ void __launch_bounds__(448, 1)
 // Tensor memory at d = 128 cannot hold a second 128-query S^T tile, so this
 // variant walks the query tiles 64 at a time and double-buffers everything:
 //   TMEM: dV [0,128), dK [128,256), S^T buffers [256,320) [320,384),
-//         dP^T buffers [384,448) [448,512); dQ^T of a step is written over that
-//         step's S^T buffer once the gradient warps have read it.
-//   SMEM: K_j, V_j resident; Q_i, dO_i, LSE_i, D_i and the P^T / dS^T operand
-//         tiles double-buffered.
+//         dP^T buffers [384,448) [448,512).  The gradient warps write P^T and
+//         dS^T (bf16, two per column) back over the start of each half's 32
+//         columns of S^T and dP^T, where dV += P^T dO and dK += dS^T Q read
+//         them as tensor-memory A operands; dQ^T of a step is then written
+//         over that step's S^T buffer.
+//   SMEM: K_j, V_j resident; Q_i, dO_i, LSE_i, D_i in three stages; dS^T
+//         (the B operand of dQ^T = K^T dS^T) double-buffered.
 // The MMA thread issues S^T(t+1) and dP^T(t+1) before it waits for the gradient
 // warps to finish step t, so the tensor core computes the next step's scores
 // while the current step's softmax gradient runs.  dQ is produced transposed,
@@ -457,14 +460,13 @@ struct BwdQ64Cfg {
   static constexpr int KV_TILE = 128 * D * 2;  // 32 KB: 2 swizzled 16 KB blocks (128 rows)
   static constexpr int Q_TILE = 64 * D * 2;    // 16 KB: 2 swizzled 8 KB blocks (64 rows)
   static constexpr int KV_BOX = 16384, Q_BOX = 8192;
-  static constexpr int OP_TILE = 128 * 64 * 2;  // P^T / dS^T: 128 keys x 64 queries, one 16 KB block
+  static constexpr int OP_TILE = 128 * 64 * 2;  // dS^T: 128 keys x 64 queries, one 16 KB block
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + KV_TILE;
   static constexpr int NST = 3;                   // Q/dO/LSE/D load stages
   static constexpr int OFF_Q = OFF_V + KV_TILE;
   static constexpr int OFF_DO = OFF_Q + NST * Q_TILE;
-  static constexpr int OFF_P = OFF_DO + NST * Q_TILE;  // 2 buffers
-  static constexpr int OFF_DS = OFF_P + 2 * OP_TILE;
+  static constexpr int OFF_DS = OFF_DO + NST * Q_TILE;  // dS^T, 2 buffers (P^T stays in TMEM)
   static constexpr int OFF_LSE = OFF_DS + 2 * OP_TILE;  // NST stages x 64 floats
   static constexpr int OFF_DV = OFF_LSE + NST * 256;
   static constexpr int OFF_BAR = OFF_DV + NST * 256;
@@ -579,7 +581,7 @@ __global__ void __launch_bounds__(448, 1)
       constexpr uint32_t id_q = make_idesc(128, 64, kFmtBF16, 1, 1);    // dQ^T: A = K^T, B = dS^T, both MN-major
       const uint32_t k_addr = smem_u32(smem + C::OFF_K), v_addr = smem_u32(smem + C::OFF_V);
       const uint32_t q_addr = smem_u32(smem + C::OFF_Q), do_addr = smem_u32(smem + C::OFF_DO);
-      const uint32_t p_addr = smem_u32(smem + C::OFF_P), ds_addr = smem_u32(smem + C::OFF_DS);
+      const uint32_t ds_addr = smem_u32(smem + C::OFF_DS);
       bool ok = mbar_wait(bar_kv, 0, abort_sh, 61);
       for (int t = 0; ok && t <= steps; ++t) {
         if (t < steps) {
@@ -620,16 +622,17 @@ __global__ void __launch_bounds__(448, 1)
           tc_fence_after();
           const int su = u % C::NST;
           const uint32_t qa = q_addr + su * C::Q_TILE, da = do_addr + su * C::Q_TILE;
-          const uint32_t pa = p_addr + b * C::OP_TILE, dsa = ds_addr + b * C::OP_TILE;
-          // dV += P^T dO_i   (M = 128 keys, N = d, K = 64 queries)
+          const uint32_t dsa = ds_addr + b * C::OP_TILE;
+          // dV += P^T dO_i   (M = 128 keys, N = d, K = 64 queries; A = P^T in TMEM, each
+          // half's 32 queries packed at the start of its own 32 columns)
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            mma_ss(tmem + C::COL_DV, make_sdesc_sw128(pa + k * 32, 16, 1024),
+            mma_ts(tmem + C::COL_DV, tmem + C::COL_S + 64 * b + (k >> 1) * 32 + (k & 1) * 8,
                    make_sdesc_sw128(da + k * 2048, C::Q_BOX, 1024), id_g, (u > 0 || k > 0) ? 1u : 0u);
-          // dK += dS^T Q_i
+          // dK += dS^T Q_i   (A = dS^T in TMEM, likewise over dP^T)
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            mma_ss(tmem + C::COL_DK, make_sdesc_sw128(dsa + k * 32, 16, 1024),
+            mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + 64 * b + (k >> 1) * 32 + (k & 1) * 8,
                    make_sdesc_sw128(qa + k * 2048, C::Q_BOX, 1024), id_g, (u > 0 || k > 0) ? 1u : 0u);
           // dQ_i^T = K_j^T dS^T   (M = d, N = 64 queries, K = 128 keys), over S^T(u)
 #pragma unroll
@@ -723,15 +726,20 @@ __global__ void __launch_bounds__(448, 1)
         dw[2 * e4] = pack_bf16x2(s01.x, s01.y);
         dw[2 * e4 + 1] = pack_bf16x2(s23.x, s23.y);
       }
+      // P^T and dS^T (bf16, two per column) over the first 16 of this half's 32
+      // columns of the S^T and dP^T buffers, whose values are in registers now:
+      // the A operands of dV += P^T dO and dK += dS^T Q
+      tmem_st16(tmem + lane_base + C::COL_S + 64 * b + half * 32, pw);
+      tmem_st16(tmem + lane_base + C::COL_DP + 64 * b + half * 32, dw);
+      // dS^T once more in SMEM: the B operand of dQ^T = K^T dS^T
       if (!(ok = mbar_wait(bar_pds_free + b, ph ^ 1, abort_sh, 68))) break;
-      uint8_t* pb = smem + C::OFF_P + b * C::OP_TILE;
       uint8_t* db = smem + C::OFF_DS + b * C::OP_TILE;
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {  // 4 chunks of 8 queries: 16-byte chunk half*4 + cc of row r
         const uint32_t off = sw128_off(r, half * 4 + cc);
-        *reinterpret_cast<uint4*>(pb + off) = make_uint4(pw[4 * cc], pw[4 * cc + 1], pw[4 * cc + 2], pw[4 * cc + 3]);
         *reinterpret_cast<uint4*>(db + off) = make_uint4(dw[4 * cc], dw[4 * cc + 1], dw[4 * cc + 2], dw[4 * cc + 3]);
       }
+      tmem_wait_st();
       tc_fence_before();
       fence_proxy_async_smem();
       mbar_arrive(bar_pds);
