@@ -38,7 +38,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 TRAFFIC = {
     "prefill": {"bytes": 811046400 + 264259840, "src": ("fwd.cuh", "sm100.cuh"),
                 "sha1": "7423259134f17bc9027b22ed228273450d627ac3"},
-    "decode": {"bytes": 1082300000, "src": ("decode.cuh", "sm100.cuh"), "sha1": "952ee5a7e1f9132f76d788fe16a32974ec02b1b2"},
+    "decode": {"bytes": 1077480000, "src": ("decode.cuh", "sm100.cuh"), "sha1": "1793d485d505f73087dea85d6b67f08fd12b9c94"},
 }
 
 
