@@ -90,7 +90,14 @@ struct FwdCfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = 2 * TILE_BYTES;
   static constexpr int OFF_V = OFF_K + NSTAGE * TILE_BYTES;
-  static constexpr int SMEM_BYTES = OFF_V + NSTAGE * TILE_BYTES + 1024;  // + alignment slack
+  // bf16 at d = 64: P goes to shared memory and PV is a shared-memory x
+  // shared-memory MMA.  With N = d = 64 an MMA reading A from tensor memory
+  // takes ~151 cycles per 16-deep step against ~108 from shared memory (at
+  // N = 128, d = 128, tensor memory is the faster, ~73).
+  static constexpr bool PV_SS = (EB == 2) && (D == 64) && !FP8P;
+  static constexpr int P_BYTES = 128 * 128 * 2;  // one 128 x 128 bf16 P tile: two 64-key boxes
+  static constexpr int OFF_P = OFF_V + NSTAGE * TILE_BYTES;
+  static constexpr int SMEM_BYTES = OFF_P + (PV_SS ? 2 * P_BYTES : 0) + 1024;  // + alignment slack
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
   static constexpr int NTHREADS = 320;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
@@ -240,6 +247,7 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t va = v_addr + s * C::TILE_BYTES;
         const uint32_t pcol = tmem + (i ? C::COL_S1 : C::COL_S0);
         const uint32_t ocol = tmem + (i ? C::COL_O1 : C::COL_O0);
+        const uint32_t pa = smem_u32(smem + C::OFF_P) + i * C::P_BYTES;
 #pragma unroll
         for (int k = 0; k < C::NK_PV; ++k) {
           // V is the MN-major B operand: 128B swizzle (bf16, E4M3) or the 32-byte-atom
@@ -248,7 +256,10 @@ __global__ void __launch_bounds__(320, 1)
                                          : make_sdesc_sw128(va + k * C::KSTEP * 128, C::BOX_BYTES, 1024);
           const uint32_t acc = (pv_count[i] > 0 || k > 0) ? 1u : 0u;
           if (!leader) continue;
-          if constexpr (C::EB == 2)
+          if constexpr (C::PV_SS)
+            mma_ss(ocol, make_sdesc_sw128(pa + (k >> 2) * (C::P_BYTES / 2) + (k & 3) * 32, 16, 1024), bd, idesc_pv,
+                   acc);
+          else if constexpr (C::EB == 2)
             mma_ts(ocol, pcol + k * 8, bd, idesc_pv, acc);
           else if constexpr (C::EB == 1)
             mma_ts_f8(ocol, pcol + k * 8, bd, idesc_pv, acc);
@@ -433,12 +444,16 @@ __global__ void __launch_bounds__(320, 1)
           }
           tmem_st32(tS, pk);
         } else if constexpr (C::EB == 2) {
+          // P in chunks of PC packed columns (2 keys each), stored as soon as each
+          // chunk is done, so that few registers besides the score row are live
+          // (measured: 16 at d = 128, 32 at d = 64)
+          constexpr int PC = D == 128 ? 16 : 32;
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t pk[32];
+          for (int h = 0; h < 64 / PC; ++h) {
+            uint32_t pk[PC];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const float2 x = ffma2(make_float2(sv[h * 64 + 2 * e], sv[h * 64 + 2 * e + 1]), c2, nm2);
+            for (int e = 0; e < PC; ++e) {
+              const float2 x = ffma2(make_float2(sv[h * 2 * PC + 2 * e], sv[h * 2 * PC + 2 * e + 1]), c2, nm2);
               const float p0 = ex2_approx(x.x);
               const float p1 = ex2_approx(x.y);
               rs4[e & 3] = fadd2(rs4[e & 3], make_float2(p0, p1));
@@ -450,7 +465,7 @@ __global__ void __launch_bounds__(320, 1)
                   if (plain_tile) {
                     fl_non += (row < N) ? 2u - __popc(nz) : 0u;
                   } else if (row < N) {
-                    const int k0 = kbase + h * 64 + 2 * e;
+                    const int k0 = kbase + h * 2 * PC + 2 * e;
                     const uint32_t f0 = (k0 <= lim && !(nz & 1u)) ? 1u : 0u;
                     const uint32_t f1 = (k0 + 1 <= lim && !(nz >> 16)) ? 1u : 0u;
                     fl_sink += (k0 < a.n_sink ? f0 : 0u) + (k0 + 1 < a.n_sink ? f1 : 0u);
@@ -461,7 +476,21 @@ __global__ void __launch_bounds__(320, 1)
                 pk[e] = pack_bf16x2(p0, p1);
               }
             }
-            tmem_st32(tS + h * 32, pk);
+            if constexpr (C::PV_SS) {
+              // keys [2 PC h, 2 PC h + 2 PC) of row r in the 64-key boxes, 128-byte swizzle
+              constexpr int CPB = 2 * PC / 8;  // 16-byte chunks per store group
+              uint8_t* pbase = smem + C::OFF_P + i * C::P_BYTES + r * 128;
+#pragma unroll
+              for (int c = 0; c < CPB; ++c) {
+                const int key8 = h * CPB + c;  // 8-key chunk index in the row (0..15)
+                *reinterpret_cast<uint4*>(pbase + (key8 >> 3) * (C::P_BYTES / 2) + (((key8 & 7) ^ (r & 7)) << 4)) =
+                    make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+              }
+            } else if constexpr (PC == 16) {
+              tmem_st16(tS + h * PC, pk);
+            } else {
+              tmem_st32(tS + h * PC, *reinterpret_cast<const uint32_t(*)[32]>(pk));
+            }
           }
         } else {
 #pragma unroll
@@ -496,6 +525,7 @@ __global__ void __launch_bounds__(320, 1)
         }
         tmem_wait_st();
         tc_fence_before();
+        if constexpr (C::PV_SS) fence_proxy_async_smem();  // P in shared memory, read by the tensor core
         mbar_arrive(&bar_p[i]);
         {
           const float2 t01 = fadd2(rs4[0], rs4[1]), t23 = fadd2(rs4[2], rs4[3]);
