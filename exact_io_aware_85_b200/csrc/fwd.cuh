@@ -446,8 +446,8 @@ __global__ void __launch_bounds__(320, 1)
         } else if constexpr (C::EB == 2) {
           // P in chunks of PC packed columns (2 keys each), stored as soon as each
           // chunk is done, so that few registers besides the score row are live
-          // (measured: 16 at d = 128, 32 at d = 64)
-          constexpr int PC = D == 128 ? 16 : 32;
+          // (measured: 8 at d = 128, 32 at d = 64)
+          constexpr int PC = D == 128 ? 8 : 32;
 #pragma unroll
           for (int h = 0; h < 64 / PC; ++h) {
             uint32_t pk[PC];
@@ -486,6 +486,8 @@ __global__ void __launch_bounds__(320, 1)
                 *reinterpret_cast<uint4*>(pbase + (key8 >> 3) * (C::P_BYTES / 2) + (((key8 & 7) ^ (r & 7)) << 4)) =
                     make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
               }
+            } else if constexpr (PC == 8) {
+              tmem_st8(tS + h * PC, pk);
             } else if constexpr (PC == 16) {
               tmem_st16(tS + h * PC, pk);
             } else {
