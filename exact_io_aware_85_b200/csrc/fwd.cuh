@@ -451,6 +451,11 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
           for (int h = 0; h < 64 / PC; ++h) {
             uint32_t pk[PC];
+            // FP8 P-cast flush counting: per pair, bit 0 / bit 16 of nz = "this P' is
+            // not zero".  Tiles without masked or sink keys only add up the flags (two
+            // 16-bit counters in one word), settled once per chunk.
+            uint32_t nzacc = 0;
+            const bool count_each = FP8P && a.stats != nullptr && !plain_tile && row < N;
 #pragma unroll
             for (int e = 0; e < PC; ++e) {
               const float2 x = ffma2(make_float2(sv[h * 2 * PC + 2 * e], sv[h * 2 * PC + 2 * e + 1]), c2, nm2);
@@ -461,20 +466,21 @@ __global__ void __launch_bounds__(320, 1)
                 uint32_t nz;
                 const float2 sp = fmul2(make_float2(p0, p1), make_float2(a.p_scale, a.p_scale));
                 pk[e] = e4m3_cast_bf16x2(sp.x, sp.y, nz);
-                if (a.stats != nullptr) {
-                  if (plain_tile) {
-                    fl_non += (row < N) ? 2u - __popc(nz) : 0u;
-                  } else if (row < N) {
-                    const int k0 = kbase + h * 2 * PC + 2 * e;
-                    const uint32_t f0 = (k0 <= lim && !(nz & 1u)) ? 1u : 0u;
-                    const uint32_t f1 = (k0 + 1 <= lim && !(nz >> 16)) ? 1u : 0u;
-                    fl_sink += (k0 < a.n_sink ? f0 : 0u) + (k0 + 1 < a.n_sink ? f1 : 0u);
-                    fl_non += (k0 < a.n_sink ? 0u : f0) + (k0 + 1 < a.n_sink ? 0u : f1);
-                  }
+                nzacc += nz;
+                if (count_each) {
+                  const int k0 = kbase + h * 2 * PC + 2 * e;
+                  const uint32_t f0 = (k0 <= lim && !(nz & 1u)) ? 1u : 0u;
+                  const uint32_t f1 = (k0 + 1 <= lim && !(nz >> 16)) ? 1u : 0u;
+                  fl_sink += (k0 < a.n_sink ? f0 : 0u) + (k0 + 1 < a.n_sink ? f1 : 0u);
+                  fl_non += (k0 < a.n_sink ? 0u : f0) + (k0 + 1 < a.n_sink ? 0u : f1);
                 }
               } else {
                 pk[e] = pack_bf16x2(p0, p1);
               }
+            }
+            if constexpr (FP8P) {
+              if (a.stats != nullptr && plain_tile && row < N)
+                fl_non += 2u * PC - ((nzacc & 0xFFFFu) + (nzacc >> 16));
             }
             if constexpr (C::PV_SS) {
               // keys [2 PC h, 2 PC h + 2 PC) of row r in the 64-key boxes, 128-byte swizzle
