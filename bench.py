@@ -3,7 +3,9 @@
 
 One step = one forward pass (fa_fwd) over one batch of synthetic input of the
 chosen workload (default: LLM prefill B=4 H=32 N=8192 d=128, bf16, causal).
-Prints one JSON line (rank 0).  See the design doc for the measurement recipe.
+Prints one JSON line (rank 0).  Timing: CUDA events on the launching stream
+around exactly K steps after W warm-up steps, inputs resident in HBM and larger
+than L2, SM clocks sampled during the timed region.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
@@ -398,7 +400,7 @@ def main():
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     peak_note = f"{peak_src} bf16 burst (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback 1590 TFLOP/s"
     if w.dtype == "fp8":
-        # no measured FP8 peak on this machine: the measured bf16 peak x the nominal 2x FP8 ratio
+        # no measured FP8 peak is available: the measured bf16 peak x the nominal 2x FP8 ratio
         peak *= 2.0
         peak_note = f"{peak_src} bf16 burst x 2 (nominal FP8/BF16 ratio)"
     bound, unit, peak_val = "tensor", "TFLOP/s", peak
