@@ -133,9 +133,10 @@ int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const
 /* One decoding step: for each query head a single new query row attends to all
  * N cached keys of its key/value head (the last row of causal attention,
  * "flash-attention-trading-models", "El algoritmo de atencion flash").  Bound by
- * reading the cache, so it runs on the CUDA cores, split over the key sequence
- * with a log-sum-exp merge of the chunks; the g = H / H_kv query heads of a
- * key/value head are served from one read of it (g <= 16).
+ * reading the cache once: split over the key sequence with a log-sum-exp merge
+ * of the chunks, K/V streamed by TMA, the per-chunk arithmetic on warp-level
+ * tensor-core MMAs; the g = H / H_kv query heads of a key/value head are served
+ * from one read of it (g <= 16).  Two launches on `stream` (split, combine). 
  * q, o: bf16 [B,H,d]; k, v: bf16 [B,H_kv,N,d]; lse: fp32 [B,H].
  * workspace: caller-owned, >= fa_decode_workspace_bytes(), 16-byte aligned. */
 size_t fa_decode_workspace_bytes(int B, int H, int H_kv, int N, int d);
