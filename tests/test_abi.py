@@ -49,6 +49,30 @@ def test_workspace_size(lib):
     assert lib.fa_bwd_workspace_bytes(1, 1, 1, 96) == 0
 
 
+def test_decode_workspace_size(lib):
+    """The decode step splits each key/value head's cache into chunks of whole
+    128-key tiles so that one wave of CTAs (one per SM of 148) covers the
+    B*H_kv heads; the workspace holds one partial O row (d floats) plus (m, l)
+    per query head and chunk, rounded up to 256 bytes."""
+    lib.fa_decode_workspace_bytes.restype = ctypes.c_size_t
+    lib.fa_decode_workspace_bytes.argtypes = [ctypes.c_int] * 5
+
+    def expect(B, H, Hkv, N, d):
+        tiles = -(-N // 128)
+        ns = min(tiles, max(1, 148 // (B * Hkv)))
+        tps = -(-tiles // ns)
+        ns = -(-tiles // tps)
+        return -(-(ns * B * H * (d + 2) * 4) // 256) * 256
+
+    for args in [(8, 32, 8, 32768, 128), (1, 8, 8, 1000, 128), (2, 32, 8, 4097, 128), (4, 16, 1, 333, 64),
+                 (1, 4, 4, 1, 64), (1, 16, 16, 70000, 128), (3, 12, 4, 65, 64), (64, 64, 8, 4096, 128)]:
+        assert lib.fa_decode_workspace_bytes(*args) == expect(*args), args
+    # the decode workload: 2 chunks of 128 tiles per key/value head
+    assert expect(8, 32, 8, 32768, 128) == 2 * 8 * 32 * 130 * 4
+    assert lib.fa_decode_workspace_bytes(1, 6, 4, 100, 128) == 0   # H not a multiple of H_kv
+    assert lib.fa_decode_workspace_bytes(1, 4, 4, 100, 96) == 0    # unsupported head dim
+
+
 def test_argument_errors_need_no_gpu(lib):
     """Validation runs before any CUDA call, so these hold on a CPU-only host."""
     vp, ci, cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
