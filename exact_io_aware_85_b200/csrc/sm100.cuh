@@ -32,8 +32,6 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-__device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
-__device__ __forceinline__ uint32_t warp_id() { return threadIdx.x >> 5; }
 
 // Status word shared by all kernels of the library.  Codes match fa_status in
 // include/fa.h; bits [8,16) carry the id of the wait that gave up.  The library
@@ -105,21 +103,6 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
 }
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
-}
-// shared -> global tiled store (bulk group completion)
-__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* smem_src, int x, int y, int z) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
-          reinterpret_cast<uint64_t>(map)),
-      "r"(smem_u32(smem_src)), "r"(x), "r"(y), "r"(z)
-      : "memory");
-}
-__device__ __forceinline__ void tma_store_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void tma_store_wait_all() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-__device__ __forceinline__ void tma_store_wait_read_all() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 // make generic-proxy shared-memory writes visible to the async proxy (TMA, tcgen05.mma)
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -271,14 +254,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -355,24 +330,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
-// E4M3 round trip of two fp32 values (round to nearest even, saturating at
-// +-448), returned as the exact fp32 values of the E4M3 results; the packed
-// bf16x2 of those values (exact: every E4M3 value is a bf16 value) is the return.
-__device__ __forceinline__ uint32_t e4m3_roundtrip_bf16x2(float lo, float hi, float& qlo, float& qhi) {
-  uint16_t e;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(e) : "f"(hi), "f"(lo));
-  uint32_t h2;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(e));
-  unsigned short hl = static_cast<unsigned short>(h2 & 0xFFFFu), hh = static_cast<unsigned short>(h2 >> 16);
-  asm("cvt.f32.f16 %0, %1;" : "=f"(qlo) : "h"(hl));
-  asm("cvt.f32.f16 %0, %1;" : "=f"(qhi) : "h"(hh));
-  return pack_bf16x2(qlo, qhi);
-}
-
-// Same cast, returned as bf16x2 bits without leaving the integer pipes for the
-// widening: E4M3 -> f16x2 is exact and every non-zero E4M3 value is an f16
-// normal, so the bf16 bits are the f16 bits shifted right by 3 with the exponent
-// rebiased (+112 << 7); zero halves stay zero.  `nz` gets bit 0 / bit 16 set for
+// E4M3 cast of two fp32 values (round to nearest even, saturating at +-448),
+// returned as bf16x2 bits without leaving the integer pipes for the widening:
+// E4M3 -> f16x2 is exact and every non-zero E4M3 value is an f16 normal, so the
+// bf16 bits are the f16 bits shifted right by 3 with the exponent rebiased
+// (+112 << 7); zero halves stay zero.  `nz` gets bit 0 / bit 16 set for
 // the halves that did not flush to zero.  Inputs must be >= 0.
 __device__ __forceinline__ uint32_t e4m3_cast_bf16x2(float lo, float hi, uint32_t& nz) {
   uint16_t e;
