@@ -38,9 +38,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # in profiles/ (fa_fwd_prefill.md, fa_decode.md); reported only while the kernel
 # sources still hash to the values they were measured with.
 TRAFFIC = {
-    "prefill": {"bytes": 808595456 + 253890048, "src": ("fwd.cuh", "sm100.cuh"),
-                "sha1": "dc9c40c1adeb517002389c3f4be53c933d55014d"},
-    "decode": {"bytes": 1077480000, "src": ("decode.cuh", "sm100.cuh"), "sha1": "9be02ee00d9793a4316f404832ad6664288e0c2f"},
+    "prefill": {"bytes": 806519296 + 252521472, "src": ("fwd.cuh", "sm100.cuh"),
+                "sha1": "032a7705e1c46488fe7ced39baa01ab1630e52bc"},
+    "decode": {"bytes": 1073831168 + 3282688, "src": ("decode.cuh", "sm100.cuh"),
+               "sha1": "8dd9914892952b31c0692bb7e820ebf9d510d600"},
 }
 
 
