@@ -80,6 +80,23 @@ def test_full_size_sampled_rows(name):
     assert np.isfinite(o).all() and np.isfinite(lse).all()
 
 
+@pytest.mark.parametrize("N,d,causal", [(131072, 128, True), (65537, 64, False)])
+def test_long_sequence_sampled_rows(N, d, causal):
+    """Long sequences (the longest 2^17 tokens; a ragged 2^16 + 1 non-causal at
+    d = 64): sampled rows, including the last tile's, against the oracle."""
+    B, H = 1, 2
+    scale = 1.0 / math.sqrt(d)
+    x = synth.make_inputs(B, H, N, d, "bf16", seed=N % 1000 + d)
+    o, lse = _run_fwd(x, B, H, N, d, causal, "bf16")
+    rows = sample_rows(B * H, N, 48, seed=2)
+    o_ref, lse_ref = oracle.attn_fwd_rows(x["q"], x["k"], x["v"], rows, causal, scale)
+    of = o.reshape(B * H, N, d)
+    lf = lse.reshape(B * H, N)
+    assert np.abs(of[rows[:, 0], rows[:, 1]] - o_ref).max() <= O_TOL
+    assert np.abs(lf[rows[:, 0], rows[:, 1]] - lse_ref).max() <= LSE_TOL
+    assert np.isfinite(o).all() and np.isfinite(lse).all()
+
+
 def test_deterministic():
     x = synth.make_inputs(1, 4, 1100, 128, "bf16", seed=3)
     a = _run_fwd(x, 1, 4, 1100, 128, True, "bf16")
