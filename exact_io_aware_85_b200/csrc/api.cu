@@ -142,7 +142,6 @@ template <int D>
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse, void* dq,
                void* dk, void* dv, int B, int H, int N, int causal, float scale, void* workspace,
                cudaStream_t stream, int Hkv = 0) {
-  using C = fa::BwdCfg<D>;
   if (Hkv <= 0) Hkv = H;
   const int BH = B * H;
   const int BHkv = B * Hkv;
@@ -182,18 +181,20 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.causal = causal ? 1 : 0;
-  if constexpr (D == 128) {
-    // pipelined 64-query variant: Q and dO tiles of 64 rows
+  if constexpr (D != 64) {
+    // 64-query variant: Q and dO tiles of 64 rows; at d = 256 two CTAs per key
+    // tile, one per 128-column slice of dV, dK and dQ
     CUtensorMap mq64, mdo64;
     if ((st = encode_qkv_map(&mq64, q, dt, 2, D, N, BH, CU_TENSOR_MAP_SWIZZLE_128B, 64)) != FA_OK) return st;
     if ((st = encode_qkv_map(&mdo64, dO, dt, 2, D, N, BH, CU_TENSOR_MAP_SWIZZLE_128B, 64)) != FA_OK) return st;
-    using CQ = fa::BwdQ64Cfg;
-    auto kern = fa::fa_bwd_main_q64_kernel;
+    using CQ = fa::BwdQ64Cfg<D>;
+    auto kern = fa::fa_bwd_main_q64_kernel<D>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, CQ::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e);
-    kern<<<static_cast<unsigned>(static_cast<long long>(n_tiles) * BHkv), CQ::NTHREADS, CQ::SMEM_BYTES, stream>>>(
-        mq64, mk, mv, mdo64, a);
+    const dim3 grid(static_cast<unsigned>(static_cast<long long>(n_tiles) * BHkv), D / 128);
+    kern<<<grid, CQ::NTHREADS, CQ::SMEM_BYTES, stream>>>(mq64, mk, mv, mdo64, a);
   } else {
+    using C = fa::BwdCfg<D>;
     auto kern = fa::fa_bwd_main_kernel<D>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e);
@@ -209,6 +210,14 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return FA_OK;
+}
+
+int launch_bwd_d(int d, const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                 void* dq, void* dk, void* dv, int B, int H, int N, int causal, float scale, void* workspace,
+                 cudaStream_t s, int Hkv = 0) {
+  if (d == 64) return launch_bwd<64>(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, causal, scale, workspace, s, Hkv);
+  if (d == 256) return launch_bwd<256>(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, causal, scale, workspace, s, Hkv);
+  return launch_bwd<128>(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, causal, scale, workspace, s, Hkv);
 }
 
 // ---------------------------------------------------------------------------
@@ -352,7 +361,7 @@ int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
 int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse, void* dq,
                void* dk, void* dv, int B, int H, int H_kv, int N, int d, int causal, float scale, void* workspace,
                size_t workspace_bytes, void* stream) {
-  int st = check_common(q, k, v, o, lse, B, H, N, d, scale);
+  int st = check_common(q, k, v, o, lse, B, H, N, d, scale, true);
   if (st != FA_OK) return st;
   if (H_kv < 1 || H % H_kv != 0) return FA_ERR_INVALID_ARG;
   if (!dO || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
@@ -360,8 +369,7 @@ int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FA_ERR_ALIGNMENT;
   if (workspace_bytes < fa_bwd_workspace_bytes(B, H, N, d)) return FA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_bwd<64>(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, causal, scale, workspace, s, H_kv)
-                 : launch_bwd<128>(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, causal, scale, workspace, s, H_kv);
+  return launch_bwd_d(d, q, k, v, o, dO, lse, dq, dk, dv, B, H, N, causal, scale, workspace, s, H_kv);
 }
 
 size_t fa_decode_workspace_bytes(int B, int H, int H_kv, int N, int d) {
@@ -475,7 +483,7 @@ int fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* sq, 
 }
 
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
-  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128 && d != 256)) return 0;
   const size_t npad = (static_cast<size_t>(N) + 127) / 128 * 128;
   const size_t bytes = static_cast<size_t>(B) * H * npad * (2 + static_cast<size_t>(d)) * sizeof(float);
   return (bytes + 255) / 256 * 256;
@@ -484,20 +492,19 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse, void* dq,
            void* dk, void* dv, int B, int H, int N, int d, int causal, float scale, void* workspace,
            size_t workspace_bytes, void* stream) {
-  int st = check_common(q, k, v, o, lse, B, H, N, d, scale);
+  int st = check_common(q, k, v, o, lse, B, H, N, d, scale, true);
   if (st != FA_OK) return st;
   if (!dO || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
   if (!aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return FA_ERR_ALIGNMENT;
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FA_ERR_ALIGNMENT;
   if (workspace_bytes < fa_bwd_workspace_bytes(B, H, N, d)) return FA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_bwd<64>(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, causal, scale, workspace, s)
-                 : launch_bwd<128>(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, causal, scale, workspace, s);
+  return launch_bwd_d(d, q, k, v, o, dO, lse, dq, dk, dv, B, H, N, causal, scale, workspace, s);
 }
 
 int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
                    void* dq, void* dk, void* dv, int B, int H, int N, int d, int causal, float scale, void* stream) {
-  int st = check_common(q, k, v, o, lse, B, H, N, d, scale);
+  int st = check_common(q, k, v, o, lse, B, H, N, d, scale, true);
   if (st != FA_OK) return st;
   if (!dO || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
   if (!aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return FA_ERR_ALIGNMENT;
@@ -505,8 +512,7 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
   void* ws = nullptr;
   if ((st = noalloc_scratch_for_current_device(&ws)) != FA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_bwd<64>(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, causal, scale, ws, s)
-                 : launch_bwd<128>(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, causal, scale, ws, s);
+  return launch_bwd_d(d, q, k, v, o, dO, lse, dq, dk, dv, B, H, N, causal, scale, ws, s);
 }
 
 int fa_watchdog_selftest(unsigned int limit_us, void* stream) {

@@ -455,15 +455,27 @@ __global__ void __launch_bounds__(448, 1)
 // while the current step's softmax gradient runs.  dQ is produced transposed,
 // dQ^T = K^T dS^T (M = d lanes, N = 64 queries), so the drain warps (thread =
 // head dimension) add into the fp32 accumulator with fully coalesced reductions.
+//
+// Head dimension 256 ("FlashAttention (IT)", section "FlashAttention-2": head
+// dimensions up to 256) does not fit this tensor-memory budget whole: dV and dK
+// of a 128-key tile alone would take all 512 columns.  Each CTA therefore owns
+// one 128-wide slice of the head dimension (blockIdx.y): S^T and dP^T contract
+// over all 256 columns (recomputed by both CTAs of a key tile), while dV, dK and
+// dQ are produced for the CTA's slice only, since dV[:, h] = P^T dO[:, h],
+// dK[:, h] = dS^T Q[:, h] and dQ[:, h] = dS K[:, h].  K and V (64 KB each) stay
+// resident; Q and dO (32 KB each per 64 queries) leave room for one load stage.
+template <int DK>
 struct BwdQ64Cfg {
-  static constexpr int D = 128;
-  static constexpr int KV_TILE = 128 * D * 2;  // 32 KB: 2 swizzled 16 KB blocks (128 rows)
-  static constexpr int Q_TILE = 64 * D * 2;    // 16 KB: 2 swizzled 8 KB blocks (64 rows)
+  static_assert(DK == 128 || DK == 256, "head dimension");
+  static constexpr int D = 128;                 // output columns of dV, dK, dQ per CTA
+  static constexpr int NBOX = DK / 64;          // 128-byte swizzled column blocks of a row
+  static constexpr int KV_TILE = 128 * DK * 2;  // NBOX swizzled 16 KB blocks (128 rows)
+  static constexpr int Q_TILE = 64 * DK * 2;    // NBOX swizzled 8 KB blocks (64 rows)
   static constexpr int KV_BOX = 16384, Q_BOX = 8192;
   static constexpr int OP_TILE = 128 * 64 * 2;  // dS^T: 128 keys x 64 queries, one 16 KB block
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + KV_TILE;
-  static constexpr int NST = 3;                   // Q/dO/LSE/D load stages
+  static constexpr int NST = DK == 128 ? 3 : 1;   // Q/dO/LSE/D load stages
   static constexpr int OFF_Q = OFF_V + KV_TILE;
   static constexpr int OFF_DO = OFF_Q + NST * Q_TILE;
   static constexpr int OFF_DS = OFF_DO + NST * Q_TILE;  // dS^T, 2 buffers (P^T stays in TMEM)
@@ -476,12 +488,14 @@ struct BwdQ64Cfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
+template <int DK>
 __global__ void __launch_bounds__(448, 1)
     fa_bwd_main_q64_kernel(const __grid_constant__ CUtensorMap tmQ64, const __grid_constant__ CUtensorMap tmK,
                            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO64,
                            const BwdArgs a) {
-  using C = BwdQ64Cfg;
+  using C = BwdQ64Cfg<DK>;
   constexpr int D = C::D;
+  const int hd = blockIdx.y;  // 128-column slice of the head dimension produced here (0 when DK = 128)
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* bar_kv = bars + 0;
@@ -549,7 +563,7 @@ __global__ void __launch_bounds__(448, 1)
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmDO64);
       mbar_arrive_expect_tx(bar_kv, 2 * C::KV_TILE);
-      for (int b = 0; b < 2; ++b) {
+      for (int b = 0; b < C::NBOX; ++b) {
         tma_load_3d(smem + C::OFF_K + b * C::KV_BOX, &tmK, bar_kv, b * 64, j * 128, bh_kv);
         tma_load_3d(smem + C::OFF_V + b * C::KV_BOX, &tmV, bar_kv, b * 64, j * 128, bh_kv);
       }
@@ -560,7 +574,7 @@ __global__ void __launch_bounds__(448, 1)
         const uint32_t ph = (t / C::NST) & 1;
         if (!mbar_wait(bar_ld_empty + s, ph ^ 1, abort_sh, 60)) break;
         mbar_arrive_expect_tx(bar_ld_full + s, 2 * C::Q_TILE + 512);
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < C::NBOX; ++b) {
           tma_load_3d(smem + C::OFF_Q + s * C::Q_TILE + b * C::Q_BOX, &tmQ64, bar_ld_full + s, b * 64, i * 64, hq);
           tma_load_3d(smem + C::OFF_DO + s * C::Q_TILE + b * C::Q_BOX, &tmDO64, bar_ld_full + s, b * 64, i * 64,
                       hq);
@@ -582,66 +596,82 @@ __global__ void __launch_bounds__(448, 1)
       const uint32_t k_addr = smem_u32(smem + C::OFF_K), v_addr = smem_u32(smem + C::OFF_V);
       const uint32_t q_addr = smem_u32(smem + C::OFF_Q), do_addr = smem_u32(smem + C::OFF_DO);
       const uint32_t ds_addr = smem_u32(smem + C::OFF_DS);
+      // dP^T(t) and S^T(t)
+      auto phase_a = [&](int t) -> bool {
+        const int b = t & 1;
+        const int st = t % C::NST;
+        if (!mbar_wait(bar_ld_full + st, (t / C::NST) & 1, abort_sh, 62)) return false;
+        tc_fence_after();
+        const uint32_t qa = q_addr + st * C::Q_TILE, da = do_addr + st * C::Q_TILE;
+        // dP^T = V_j dO_i^T first: its buffer was released when step t-2's
+        // gradient finished, so the tensor core has work while the dQ drain of
+        // step t-2 empties the S^T buffer
+#pragma unroll
+        for (int k = 0; k < DK / 16; ++k) {
+          const uint32_t va = v_addr + (k >> 2) * C::KV_BOX + (k & 3) * 32;
+          const uint32_t db = da + (k >> 2) * C::Q_BOX + (k & 3) * 32;
+          mma_ss(tmem + C::COL_DP + 64 * b, make_sdesc_sw128(va, 16, 1024), make_sdesc_sw128(db, 16, 1024), id_s,
+                 k > 0);
+        }
+        mma_commit(bar_dp_full + b);
+        if (t >= 2) {
+          if (!mbar_wait(bar_dq_free + b, ((t - 2) >> 1) & 1, abort_sh, 63)) return false;
+          tc_fence_after();
+        }
+        // S^T = K_j Q_i^T   (M = 128 keys, N = 64 queries, K = d), over dQ^T(t-2)
+#pragma unroll
+        for (int k = 0; k < DK / 16; ++k) {
+          const uint32_t ka = k_addr + (k >> 2) * C::KV_BOX + (k & 3) * 32;
+          const uint32_t qb = qa + (k >> 2) * C::Q_BOX + (k & 3) * 32;
+          mma_ss(tmem + C::COL_S + 64 * b, make_sdesc_sw128(ka, 16, 1024), make_sdesc_sw128(qb, 16, 1024), id_s,
+                 k > 0);
+        }
+        mma_commit(bar_s_full + b);
+        return true;
+      };
+      // dV(u), dK(u), dQ^T(u) once the gradient warps have written P^T and dS^T
+      auto phase_b = [&](int u) -> bool {
+        const int b = u & 1;
+        if (!mbar_wait(bar_pds, u & 1, abort_sh, 64)) return false;
+        tc_fence_after();
+        const int su = u % C::NST;
+        // this CTA's slice of the head dimension: blocks 2 hd and 2 hd + 1
+        const uint32_t qa = q_addr + su * C::Q_TILE + hd * 2 * C::Q_BOX;
+        const uint32_t da = do_addr + su * C::Q_TILE + hd * 2 * C::Q_BOX;
+        const uint32_t kh = k_addr + hd * 2 * C::KV_BOX;
+        const uint32_t dsa = ds_addr + b * C::OP_TILE;
+        // dV += P^T dO_i   (M = 128 keys, N = 128 columns, K = 64 queries; A = P^T in
+        // TMEM, each half's 32 queries packed at the start of its own 32 columns)
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          mma_ts(tmem + C::COL_DV, tmem + C::COL_S + 64 * b + (k >> 1) * 32 + (k & 1) * 8,
+                 make_sdesc_sw128(da + k * 2048, C::Q_BOX, 1024), id_g, (u > 0 || k > 0) ? 1u : 0u);
+        // dK += dS^T Q_i   (A = dS^T in TMEM, likewise over dP^T)
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + 64 * b + (k >> 1) * 32 + (k & 1) * 8,
+                 make_sdesc_sw128(qa + k * 2048, C::Q_BOX, 1024), id_g, (u > 0 || k > 0) ? 1u : 0u);
+        // dQ_i^T = K_j^T dS^T   (M = 128 columns, N = 64 queries, K = 128 keys), over S^T(u)
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          mma_ss(tmem + C::COL_S + 64 * b, make_sdesc_sw128(kh + k * 2048, C::KV_BOX, 1024),
+                 make_sdesc_sw128(dsa + k * 2048, C::KV_BOX, 1024), id_q, k > 0 ? 1u : 0u);
+        mma_commit(bar_dq_full + b);
+        mma_commit(bar_ld_empty + su);
+        mma_commit(bar_pds_free + b);
+        return true;
+      };
       bool ok = mbar_wait(bar_kv, 0, abort_sh, 61);
       for (int t = 0; ok && t <= steps; ++t) {
-        if (t < steps) {
-          const int b = t & 1;
-          const int st = t % C::NST;
-          if (!(ok = mbar_wait(bar_ld_full + st, (t / C::NST) & 1, abort_sh, 62))) break;
-          tc_fence_after();
-          const uint32_t qa = q_addr + st * C::Q_TILE, da = do_addr + st * C::Q_TILE;
-          // dP^T = V_j dO_i^T first: its buffer was released when step t-2's
-          // gradient finished, so the tensor core has work while the dQ drain of
-          // step t-2 empties the S^T buffer
-#pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint32_t va = v_addr + (k >> 2) * C::KV_BOX + (k & 3) * 32;
-            const uint32_t db = da + (k >> 2) * C::Q_BOX + (k & 3) * 32;
-            mma_ss(tmem + C::COL_DP + 64 * b, make_sdesc_sw128(va, 16, 1024), make_sdesc_sw128(db, 16, 1024), id_s,
-                   k > 0);
-          }
-          mma_commit(bar_dp_full + b);
-          if (t >= 2) {
-            if (!(ok = mbar_wait(bar_dq_free + b, ((t - 2) >> 1) & 1, abort_sh, 63))) break;
-            tc_fence_after();
-          }
-          // S^T = K_j Q_i^T   (M = 128 keys, N = 64 queries, K = d), over dQ^T(t-2)
-#pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint32_t ka = k_addr + (k >> 2) * C::KV_BOX + (k & 3) * 32;
-            const uint32_t qb = qa + (k >> 2) * C::Q_BOX + (k & 3) * 32;
-            mma_ss(tmem + C::COL_S + 64 * b, make_sdesc_sw128(ka, 16, 1024), make_sdesc_sw128(qb, 16, 1024), id_s,
-                   k > 0);
-          }
-          mma_commit(bar_s_full + b);
-        }
-        if (t >= 1) {
-          const int u = t - 1;
-          const int b = u & 1;
-          if (!(ok = mbar_wait(bar_pds, u & 1, abort_sh, 64))) break;
-          tc_fence_after();
-          const int su = u % C::NST;
-          const uint32_t qa = q_addr + su * C::Q_TILE, da = do_addr + su * C::Q_TILE;
-          const uint32_t dsa = ds_addr + b * C::OP_TILE;
-          // dV += P^T dO_i   (M = 128 keys, N = d, K = 64 queries; A = P^T in TMEM, each
-          // half's 32 queries packed at the start of its own 32 columns)
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_ts(tmem + C::COL_DV, tmem + C::COL_S + 64 * b + (k >> 1) * 32 + (k & 1) * 8,
-                   make_sdesc_sw128(da + k * 2048, C::Q_BOX, 1024), id_g, (u > 0 || k > 0) ? 1u : 0u);
-          // dK += dS^T Q_i   (A = dS^T in TMEM, likewise over dP^T)
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + 64 * b + (k >> 1) * 32 + (k & 1) * 8,
-                   make_sdesc_sw128(qa + k * 2048, C::Q_BOX, 1024), id_g, (u > 0 || k > 0) ? 1u : 0u);
-          // dQ_i^T = K_j^T dS^T   (M = d, N = 64 queries, K = 128 keys), over S^T(u)
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            mma_ss(tmem + C::COL_S + 64 * b, make_sdesc_sw128(k_addr + k * 2048, C::KV_BOX, 1024),
-                   make_sdesc_sw128(dsa + k * 2048, C::KV_BOX, 1024), id_q, k > 0 ? 1u : 0u);
-          mma_commit(bar_dq_full + b);
-          mma_commit(bar_ld_empty + su);
-          mma_commit(bar_pds_free + b);
+        if constexpr (C::NST > 1) {
+          // the next step's scores are issued before this step's gradient is awaited
+          if (t < steps && !(ok = phase_a(t))) break;
+          if (t >= 1 && !(ok = phase_b(t - 1))) break;
+        } else {
+          // one load stage: Q_i and dO_i of step t arrive only after step t-1's
+          // last reader of the stage (dK) has been issued and has finished
+          if (t >= 1 && !(ok = phase_b(t - 1))) break;
+          if (t < steps && !(ok = phase_a(t))) break;
         }
       }
       if (ok) mma_commit(bar_acc);
@@ -663,9 +693,9 @@ __global__ void __launch_bounds__(448, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bar_dq_free + b);  // the buffer is free as soon as it is in registers
-      float* dst = a.dq_acc + (static_cast<size_t>(hq) * a.Npad + static_cast<size_t>(i) * 64) * D + c;
+      float* dst = a.dq_acc + (static_cast<size_t>(hq) * a.Npad + static_cast<size_t>(i) * 64) * DK + hd * 128 + c;
 #pragma unroll
-      for (int q = 0; q < 64; ++q) atomicAdd(dst + static_cast<size_t>(q) * D, __uint_as_float(v[q]));
+      for (int q = 0; q < 64; ++q) atomicAdd(dst + static_cast<size_t>(q) * DK, __uint_as_float(v[q]));
     }
   } else {
     // ============================ gradient warps =============================
@@ -749,7 +779,7 @@ __global__ void __launch_bounds__(448, 1)
     if (ok) {
       tc_fence_after();
       const uint32_t col = half ? C::COL_DK : C::COL_DV;
-      __nv_bfloat16* dst = (half ? a.dk : a.dv) + (static_cast<size_t>(bh_kv) * N + key) * D;
+      __nv_bfloat16* dst = (half ? a.dk : a.dv) + (static_cast<size_t>(bh_kv) * N + key) * DK + hd * 128;
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t v[32];

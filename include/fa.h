@@ -14,8 +14,9 @@
  *    device arrays (the (batch, heads, seq, head_dim) layout of the pages'
  *    framework example); lse is a contiguous [B, H, N] float32 device array.
  *    LSE is the natural-log logsumexp of the scaled scores of each query row.
- *  - Sizes: B >= 1, H >= 1, N >= 1, d in {64, 128} (fa_fwd and fa_fwd_gqa also
- *    take d = 256, "FlashAttention (IT)", "FlashAttention-2"); B*H*N*d < 2^31.
+ *  - Sizes: B >= 1, H >= 1, N >= 1, d in {64, 128} (fa_fwd, fa_fwd_gqa, fa_bwd,
+ *    fa_bwd_gqa and fa_bwd_noalloc also take d = 256, "FlashAttention (IT)",
+ *    "FlashAttention-2"); B*H*N*d < 2^31.
  *  - scale: the softmax scale (usually 1/sqrt(d)); finite and > 0.
  *  - causal != 0: query i attends to keys j <= i (square, top-left aligned);
  *    tiles that lie entirely in the future are skipped, never loaded.

@@ -46,6 +46,7 @@ def test_workspace_size(lib):
     lib.fa_bwd_workspace_bytes.argtypes = [ctypes.c_int] * 4
     assert lib.fa_bwd_workspace_bytes(2, 16, 4096, 128) == 2 * 16 * 4096 * 130 * 4
     assert lib.fa_bwd_workspace_bytes(1, 1, 1, 64) == 128 * 66 * 4
+    assert lib.fa_bwd_workspace_bytes(1, 1, 1, 256) == 128 * 258 * 4
     assert lib.fa_bwd_workspace_bytes(1, 1, 1, 96) == 0
 
 

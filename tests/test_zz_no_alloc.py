@@ -52,6 +52,7 @@ def _case(B, H, N, d, causal, seed):
 def test_noalloc_matches_fa_bwd_on_two_calls_in_a_row():
     _case(1, 2, 700, 128, True, seed=901)   # first call on this device sets up the scratch address
     _case(2, 1, 257, 64, False, seed=902)   # second call reuses the array left by the first
+    _case(1, 2, 300, 256, True, seed=903)   # head dimension 256 (two CTAs per key tile)
 
 
 def test_noalloc_refuses_sizes_beyond_the_scratch_array():
