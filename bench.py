@@ -411,7 +411,8 @@ def main():
         peak_val = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
         peak_note = f"{peak_src} HBM copy bandwidth (MEASURED_PEAKS.json)"
     if w.backward:
-        kernel_name = "training step: fa_fwd_kernel<bf16,%d> + fa_bwd (pre, main, post)" % w.d
+        kernel_name = "training step: %s + fa_bwd (pre, main, post)" % (
+            "fa_fwd256_kernel" if w.d == 256 else "fa_fwd_kernel<bf16,%d>" % w.d)
     elif w.sink:
         kernel_name = "fa_fwd_kernel<bf16,%d,FP8P>" % w.d
     elif w.dtype == "fp8":

@@ -463,7 +463,11 @@ __global__ void __launch_bounds__(448, 1)
 // over all 256 columns (recomputed by both CTAs of a key tile), while dV, dK and
 // dQ are produced for the CTA's slice only, since dV[:, h] = P^T dO[:, h],
 // dK[:, h] = dS^T Q[:, h] and dQ[:, h] = dS K[:, h].  K and V (64 KB each) stay
-// resident; Q and dO (32 KB each per 64 queries) leave room for one load stage.
+// resident; Q and dO (32 KB each per 64 queries) leave room for one load stage,
+// filled in two halves with barriers of their own: the other slice's columns
+// (read by S^T and dP^T only) are refilled as soon as those two are done, while
+// the gradient and dV/dK/dQ of the step still run; this CTA's slice follows once
+// dK has finished with it.  The scores of the next step start on the early half.
 template <int DK>
 struct BwdQ64Cfg {
   static_assert(DK == 128 || DK == 256, "head dimension");
@@ -534,7 +538,8 @@ __global__ void __launch_bounds__(448, 1)
   if (threadIdx.x == 0) {
     *abort_sh = 0;
     mbar_init(bar_kv, 1);
-    for (int b = 0; b < C::NST; ++b) {
+    // DK = 256 fills its single stage in two halves, one slot each
+    for (int b = 0; b < (C::NST > 1 ? C::NST : 2); ++b) {
       mbar_init(bar_ld_full + b, 1);
       mbar_init(bar_ld_empty + b, 1);
     }
@@ -568,24 +573,54 @@ __global__ void __launch_bounds__(448, 1)
         tma_load_3d(smem + C::OFF_V + b * C::KV_BOX, &tmV, bar_kv, b * 64, j * 128, bh_kv);
       }
       int t = 0;
-      for (; t < steps; ++t) {
-        const int i = step_tile(t), hq = step_head(t);
-        const int s = t % C::NST;
-        const uint32_t ph = (t / C::NST) & 1;
-        if (!mbar_wait(bar_ld_empty + s, ph ^ 1, abort_sh, 60)) break;
-        mbar_arrive_expect_tx(bar_ld_full + s, 2 * C::Q_TILE + 512);
-        for (int b = 0; b < C::NBOX; ++b) {
-          tma_load_3d(smem + C::OFF_Q + s * C::Q_TILE + b * C::Q_BOX, &tmQ64, bar_ld_full + s, b * 64, i * 64, hq);
-          tma_load_3d(smem + C::OFF_DO + s * C::Q_TILE + b * C::Q_BOX, &tmDO64, bar_ld_full + s, b * 64, i * 64,
-                      hq);
+      if constexpr (DK == 256) {
+        // one stage in two halves: slot 1 = the other slice's blocks, slot 0 =
+        // this CTA's slice plus the row statistics
+        const int ho = 1 - hd;
+        int n_early = 0;
+        for (; t < steps; ++t) {
+          const int i = step_tile(t), hq = step_head(t);
+          const uint32_t ph = t & 1;
+          if (!mbar_wait(bar_ld_empty + 1, ph ^ 1, abort_sh, 70)) break;
+          mbar_arrive_expect_tx(bar_ld_full + 1, 4 * C::Q_BOX);
+          for (int b = 2 * ho; b < 2 * ho + 2; ++b) {
+            tma_load_3d(smem + C::OFF_Q + b * C::Q_BOX, &tmQ64, bar_ld_full + 1, b * 64, i * 64, hq);
+            tma_load_3d(smem + C::OFF_DO + b * C::Q_BOX, &tmDO64, bar_ld_full + 1, b * 64, i * 64, hq);
+          }
+          n_early = t + 1;
+          if (!mbar_wait(bar_ld_empty, ph ^ 1, abort_sh, 60)) break;
+          mbar_arrive_expect_tx(bar_ld_full, 4 * C::Q_BOX + 512);
+          for (int b = 2 * hd; b < 2 * hd + 2; ++b) {
+            tma_load_3d(smem + C::OFF_Q + b * C::Q_BOX, &tmQ64, bar_ld_full, b * 64, i * 64, hq);
+            tma_load_3d(smem + C::OFF_DO + b * C::Q_BOX, &tmDO64, bar_ld_full, b * 64, i * 64, hq);
+          }
+          const size_t roff = static_cast<size_t>(hq) * a.Npad + static_cast<size_t>(i) * 64;
+          bulk_load(smem + C::OFF_LSE, a.lse2 + roff, 256, bar_ld_full);
+          bulk_load(smem + C::OFF_DV, a.dvec + roff, 256, bar_ld_full);
         }
-        const size_t roff = static_cast<size_t>(hq) * a.Npad + static_cast<size_t>(i) * 64;
-        bulk_load(smem + C::OFF_LSE + s * 256, a.lse2 + roff, 256, bar_ld_full + s);
-        bulk_load(smem + C::OFF_DV + s * 256, a.dvec + roff, 256, bar_ld_full + s);
+        mbar_wait_drain(bar_kv, 0, 100000000ull);
+        if (n_early > 0) mbar_wait_drain(bar_ld_full + 1, (n_early - 1) & 1, 100000000ull);
+        if (t > 0) mbar_wait_drain(bar_ld_full, (t - 1) & 1, 100000000ull);
+      } else {
+        for (; t < steps; ++t) {
+          const int i = step_tile(t), hq = step_head(t);
+          const int s = t % C::NST;
+          const uint32_t ph = (t / C::NST) & 1;
+          if (!mbar_wait(bar_ld_empty + s, ph ^ 1, abort_sh, 60)) break;
+          mbar_arrive_expect_tx(bar_ld_full + s, 2 * C::Q_TILE + 512);
+          for (int b = 0; b < C::NBOX; ++b) {
+            tma_load_3d(smem + C::OFF_Q + s * C::Q_TILE + b * C::Q_BOX, &tmQ64, bar_ld_full + s, b * 64, i * 64, hq);
+            tma_load_3d(smem + C::OFF_DO + s * C::Q_TILE + b * C::Q_BOX, &tmDO64, bar_ld_full + s, b * 64, i * 64,
+                        hq);
+          }
+          const size_t roff = static_cast<size_t>(hq) * a.Npad + static_cast<size_t>(i) * 64;
+          bulk_load(smem + C::OFF_LSE + s * 256, a.lse2 + roff, 256, bar_ld_full + s);
+          bulk_load(smem + C::OFF_DV + s * 256, a.dvec + roff, 256, bar_ld_full + s);
+        }
+        mbar_wait_drain(bar_kv, 0, 100000000ull);
+        for (int u = max(0, t - C::NST); u < t; ++u)
+          mbar_wait_drain(bar_ld_full + u % C::NST, (u / C::NST) & 1, 100000000ull);
       }
-      mbar_wait_drain(bar_kv, 0, 100000000ull);
-      for (int u = max(0, t - C::NST); u < t; ++u)
-        mbar_wait_drain(bar_ld_full + u % C::NST, (u / C::NST) & 1, 100000000ull);
     }
   } else if (warp == 13) {
     // ============================ MMA issuer =================================
@@ -596,8 +631,51 @@ __global__ void __launch_bounds__(448, 1)
       const uint32_t k_addr = smem_u32(smem + C::OFF_K), v_addr = smem_u32(smem + C::OFF_V);
       const uint32_t q_addr = smem_u32(smem + C::OFF_Q), do_addr = smem_u32(smem + C::OFF_DO);
       const uint32_t ds_addr = smem_u32(smem + C::OFF_DS);
+      // dP^T(t) and S^T(t) at DK = 256: the other slice's half of Q_i and dO_i
+      // (slot 1) first, this CTA's slice (slot 0) last
+      auto phase_a2 = [&](int t) -> bool {
+        const int b = t & 1;
+        const int ho = 1 - hd;
+        auto dp_steps = [&](int h, bool first) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const int k = 8 * h + kk;
+            const uint32_t va = v_addr + (k >> 2) * C::KV_BOX + (k & 3) * 32;
+            const uint32_t db = do_addr + (k >> 2) * C::Q_BOX + (k & 3) * 32;
+            mma_ss(tmem + C::COL_DP + 64 * b, make_sdesc_sw128(va, 16, 1024), make_sdesc_sw128(db, 16, 1024), id_s,
+                   (first && kk == 0) ? 0u : 1u);
+          }
+        };
+        auto s_steps = [&](int h, bool first) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const int k = 8 * h + kk;
+            const uint32_t ka = k_addr + (k >> 2) * C::KV_BOX + (k & 3) * 32;
+            const uint32_t qb = q_addr + (k >> 2) * C::Q_BOX + (k & 3) * 32;
+            mma_ss(tmem + C::COL_S + 64 * b, make_sdesc_sw128(ka, 16, 1024), make_sdesc_sw128(qb, 16, 1024), id_s,
+                   (first && kk == 0) ? 0u : 1u);
+          }
+        };
+        if (!mbar_wait(bar_ld_full + 1, t & 1, abort_sh, 71)) return false;
+        tc_fence_after();
+        dp_steps(ho, true);
+        if (t >= 2) {
+          if (!mbar_wait(bar_dq_free + b, ((t - 2) >> 1) & 1, abort_sh, 63)) return false;
+          tc_fence_after();
+        }
+        s_steps(ho, true);
+        if (!mbar_wait(bar_ld_full, t & 1, abort_sh, 62)) return false;
+        tc_fence_after();
+        s_steps(hd, false);
+        mma_commit(bar_s_full + b);
+        dp_steps(hd, false);
+        mma_commit(bar_dp_full + b);
+        mma_commit(bar_ld_empty + 1);  // the other slice's half is read by nothing else
+        return true;
+      };
       // dP^T(t) and S^T(t)
       auto phase_a = [&](int t) -> bool {
+        if constexpr (DK == 256) return phase_a2(t);
         const int b = t & 1;
         const int st = t % C::NST;
         if (!mbar_wait(bar_ld_full + st, (t / C::NST) & 1, abort_sh, 62)) return false;

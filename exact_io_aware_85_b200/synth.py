@@ -68,6 +68,8 @@ WORKLOADS = {
     "prefill_d256": Workload("prefill_d256", 4, 16, 8192, 256, "bf16", True),
     # one decoding step of 8 sequences against a 32K-token key/value cache, 8 KV heads
     "decode": Workload("decode", 8, 32, 32768, 128, "bf16", False, hkv=8, decode=True),
+    # a training step at head dim 256 (forward + backward), 8192 tokens
+    "train_d256": Workload("train_d256", 2, 8, 8192, 256, "bf16", True, backward=True),
 }
 
 SINK_DELTAS = (0.0, 2.0, 4.0, 6.0, 7.0, 8.0, 10.0, 12.0)
