@@ -373,7 +373,7 @@ int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const
 }
 
 size_t fa_decode_workspace_bytes(int B, int H, int H_kv, int N, int d) {
-  if (B < 1 || H < 1 || H_kv < 1 || N < 1 || H % H_kv != 0 || (d != 64 && d != 128)) return 0;
+  if (B < 1 || H < 1 || H_kv < 1 || N < 1 || H % H_kv != 0 || (d != 64 && d != 128 && d != 256)) return 0;
   int ns, tps;
   decode_plan(B, H_kv, N, &ns, &tps);
   const size_t bytes = static_cast<size_t>(ns) * B * H * (static_cast<size_t>(d) + 2) * sizeof(float);
@@ -385,7 +385,7 @@ int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, 
   if (!q || !k || !v || !o || !lse || !workspace) return FA_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || H_kv < 1 || N < 1 || H % H_kv != 0) return FA_ERR_INVALID_ARG;
   if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
   const int g = H / H_kv;
   if (g > fa::kDecMaxG) return FA_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * H_kv * N * d >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
@@ -417,10 +417,14 @@ int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, 
     e = g <= 8 ? launch_decode_split<64, 1>(grid, s, mk, mv, a) : launch_decode_split<64, 2>(grid, s, mk, mv, a);
     if (e != cudaSuccess) return cuda_fail(e);
     fa::fa_decode_combine_kernel<64><<<B * H, 64, 0, s>>>(a);
-  } else {
+  } else if (d == 128) {
     e = g <= 8 ? launch_decode_split<128, 1>(grid, s, mk, mv, a) : launch_decode_split<128, 2>(grid, s, mk, mv, a);
     if (e != cudaSuccess) return cuda_fail(e);
     fa::fa_decode_combine_kernel<128><<<B * H, 128, 0, s>>>(a);
+  } else {
+    e = g <= 8 ? launch_decode_split<256, 1>(grid, s, mk, mv, a) : launch_decode_split<256, 2>(grid, s, mk, mv, a);
+    if (e != cudaSuccess) return cuda_fail(e);
+    fa::fa_decode_combine_kernel<256><<<B * H, 256, 0, s>>>(a);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);

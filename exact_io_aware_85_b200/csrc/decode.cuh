@@ -20,6 +20,9 @@
 //                      (m16n8k16, bf16 in, fp32 accumulate):
 //                        S^T = K Q^T      warp w: keys [16w, 16w + 16)
 //                        O^T += V^T P^T   warp w: 16 of the d output columns
+//                      At d = 256 a K or V tile is 64 KB, so the ring holds
+//                      single tiles (K_i, V_i, K_i+1, ...), each refilled as
+//                      soon as it is consumed: still 128-192 KB in flight.
 //                      Out of a streaming kernel the tensor cores take the
 //                      instruction count, not the time: on the CUDA cores the
 //                      same arithmetic left the kernel issue-latency bound at
@@ -54,8 +57,9 @@ template <int D>
 struct DecodeLayout {
   static constexpr int BOX = kDecKT * 128;          // 128 rows x 128 B (64 columns)
   static constexpr int TILE = (D / 64) * BOX;       // one 128 x D tile
-  static constexpr int STAGE = 2 * TILE;            // K then V
-  static constexpr int STAGES = 196608 / STAGE;     // 192 KB ring: 3 stages (d 128), 6 (d 64)
+  static constexpr bool SPLIT_KV = D > 128;         // ring slots hold one tile (K or V), not a K+V pair
+  static constexpr int STAGE = SPLIT_KV ? TILE : 2 * TILE;
+  static constexpr int STAGES = 196608 / STAGE;     // 192 KB ring: 3 stages (d 128), 6 (d 64), 3 tiles (d 256)
   static constexpr int P_LD = kDecKT * 2 + 16;      // bytes per P^T row
   static constexpr int OFF_P = STAGES * STAGE;
   static constexpr int OFF_RED = OFF_P + kDecMaxG * P_LD;  // float [2][8 warps][16]
@@ -118,20 +122,38 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     fence_mbar_init();
   }
   __syncthreads();
-  auto issue = [&](int i) {  // tile t0 + i into stage i % NST
-    uint8_t* st = smem + (i % NST) * L::STAGE;
-    uint64_t* bar = &full[i % NST];
+  // ring loads: K+V of tile t0 + n (d <= 128), or K (n even) / V (n odd) of tile
+  // t0 + n/2 (d = 256), into slot n % NST; only thread 0 issues and counts them
+  const int n_loads = L::SPLIT_KV ? 2 * nt : nt;
+  int issued = 0;
+  auto issue = [&](int n) {
+    uint8_t* st = smem + (n % NST) * L::STAGE;
+    uint64_t* bar = &full[n % NST];
     mbar_arrive_expect_tx(bar, L::STAGE);
-    const int key0 = (t0 + i) * kDecKT;
-    for (int b = 0; b < D / 64; ++b) {
-      tma_load_3d(st + b * L::BOX, &tmK, bar, b * 64, key0, bhkv);
-      tma_load_3d(st + L::TILE + b * L::BOX, &tmV, bar, b * 64, key0, bhkv);
+    if constexpr (L::SPLIT_KV) {
+      const int key0 = (t0 + n / 2) * kDecKT;
+      for (int b = 0; b < D / 64; ++b) {
+        if (n & 1) tma_load_3d(st + b * L::BOX, &tmV, bar, b * 64, key0, bhkv);
+        else tma_load_3d(st + b * L::BOX, &tmK, bar, b * 64, key0, bhkv);
+      }
+    } else {
+      const int key0 = (t0 + n) * kDecKT;
+      for (int b = 0; b < D / 64; ++b) {
+        tma_load_3d(st + b * L::BOX, &tmK, bar, b * 64, key0, bhkv);
+        tma_load_3d(st + L::TILE + b * L::BOX, &tmV, bar, b * 64, key0, bhkv);
+      }
     }
+    issued = n + 1;
+  };
+  // let every copy still in flight land before the block can exit
+  auto drain_from = [&](int n0) {
+    if (tid == 0)
+      for (int n = n0; n < issued; ++n) mbar_wait_drain(&full[n % NST], (n / NST) & 1, 100000000ull);
   };
   if (tid == 0) {
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
-    for (int i = 0; i < NST && i < nt; ++i) issue(i);
+    for (int n = 0; n < NST && n < n_loads; ++n) issue(n);
   }
 
   // Q^T as the B operand of S^T = K Q^T: for query column n = 8j + grp and
@@ -151,30 +173,31 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   // per thread: query columns 8j + 2tq and 8j + 2tq + 1 (the same in the score
   // and the output fragments)
   float m_run[NT][2], l_run[NT][2];
-  float oacc[NT][4];
+  // output columns of this warp: MT blocks of 16 (two at d = 256), and, for
+  // d = 64, its half of each tile's keys
+  constexpr int MT = D > 128 ? 2 : 1;
+  constexpr int WARPS_PER_D = D / (16 * MT);           // 8 (d 256, 128) or 4 (d 64)
+  float oacc[NT][MT][4];
 #pragma unroll
   for (int j = 0; j < NT; ++j) {
     m_run[j][0] = m_run[j][1] = -INFINITY;
     l_run[j][0] = l_run[j][1] = 0.f;
-    oacc[j][0] = oacc[j][1] = oacc[j][2] = oacc[j][3] = 0.f;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) oacc[j][mt][0] = oacc[j][mt][1] = oacc[j][mt][2] = oacc[j][mt][3] = 0.f;
   }
-  // output columns of this warp and, for d = 64, its half of each tile's keys
-  constexpr int WARPS_PER_D = D / 16;                  // 8 (d 128) or 4 (d 64)
-  const int ocol = 16 * (warp % WARPS_PER_D);
+  const int ocol = 16 * MT * (warp % WARPS_PER_D);
   const int khalf = warp / WARPS_PER_D;                // 0, or 0/1 for d 64
   constexpr int PV_STEPS = (kDecKT / 16) / (8 / WARPS_PER_D);
   const uint32_t pt_addr = smem_u32(pt);
   bool ok = true;
 
   for (int i = 0; i < nt; ++i) {
-    const int st_i = i % NST;
-    const uint32_t kt = smem_u32(smem + st_i * L::STAGE);
-    const uint32_t vt = kt + L::TILE;
-    const bool got = mbar_wait(&full[st_i], (i / NST) & 1, abort_sh, 20);
+    const int nk = L::SPLIT_KV ? 2 * i : i;  // the load that holds K_i
+    const uint32_t kt = smem_u32(smem + (nk % NST) * L::STAGE);
+    const uint32_t vt = L::SPLIT_KV ? smem_u32(smem + ((nk + 1) % NST) * L::STAGE) : kt + L::TILE;
+    const bool got = mbar_wait(&full[nk % NST], (nk / NST) & 1, abort_sh, 20);
     if (__syncthreads_or(!got)) {
-      // let the copies still in flight land before the block can exit
-      if (tid == 0)
-        for (int j = i; j < min(nt, i + NST); ++j) mbar_wait_drain(&full[j % NST], (j / NST) & 1, 100000000ull);
+      drain_from(nk);
       ok = false;
       break;
     }
@@ -220,8 +243,16 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       }
     }
     __syncthreads();
-    // the previous tile's stage is free now (every warp is past its PV)
-    if (tid == 0 && i > 0 && i - 1 + NST < nt) issue(i - 1 + NST);
+    if constexpr (L::SPLIT_KV) {
+      // every warp is past PV(i-1) and S^T(i): the slots of V_{i-1} and K_i refill
+      if (tid == 0) {
+        if (i > 0 && 2 * i + 2 < n_loads) issue(2 * i + 2);
+        if (2 * i + 3 < n_loads) issue(2 * i + 3);
+      }
+    } else {
+      // the previous tile's stage is free now (every warp is past its PV)
+      if (tid == 0 && i > 0 && i - 1 + NST < nt) issue(i - 1 + NST);
+    }
     float alpha[NT][2];
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
@@ -255,7 +286,17 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         red_sum[warp * kDecMaxG + n0 + 1] = s1;
       }
     }
-    __syncthreads();
+    if constexpr (L::SPLIT_KV) {
+      // V_i has its own slot and barrier
+      const bool got_v = mbar_wait(&full[(nk + 1) % NST], ((nk + 1) / NST) & 1, abort_sh, 21);
+      if (__syncthreads_or(!got_v)) {
+        drain_from(nk + 1);
+        ok = false;
+        break;
+      }
+    } else {
+      __syncthreads();
+    }
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
 #pragma unroll
@@ -266,27 +307,35 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         for (int w = 0; w < 8; ++w) sum += red_sum[w * kDecMaxG + n];
         l_run[j][c] = l_run[j][c] * alpha[j][c] + sum;
       }
-      oacc[j][0] *= alpha[j][0];
-      oacc[j][1] *= alpha[j][1];
-      oacc[j][2] *= alpha[j][0];
-      oacc[j][3] *= alpha[j][1];
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        oacc[j][mt][0] *= alpha[j][0];
+        oacc[j][mt][1] *= alpha[j][1];
+        oacc[j][mt][2] *= alpha[j][0];
+        oacc[j][mt][3] *= alpha[j][1];
+      }
     }
-    // ---- O^T += V^T P^T for output columns [ocol, ocol + 16) ----------------------
+    // ---- O^T += V^T P^T for output columns [ocol, ocol + 16 MT) -----------------
     {
       const int mi = lane >> 3, r8 = lane & 7;
-      const int box = ocol / 64;
-      const int cbase = (ocol % 64) / 8 + (mi & 1);  // 16-byte chunk of the 8 columns
 #pragma unroll
       for (int s = 0; s < PV_STEPS; ++s) {
         const int kk = khalf * PV_STEPS + s;           // 16-key step
         const int vrow = 16 * kk + r8 + 8 * (mi >> 1);
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4_t(vt + box * L::BOX + vrow * 128 + ((cbase ^ (vrow & 7)) << 4), a0, a1, a2, a3);
+        uint32_t av[MT][4];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          const int col = ocol + 16 * mt;
+          const int cbase = (col % 64) / 8 + (mi & 1);  // 16-byte chunk of the 8 columns
+          ldsm_x4_t(vt + (col / 64) * L::BOX + vrow * 128 + ((cbase ^ (vrow & 7)) << 4), av[mt][0], av[mt][1],
+                    av[mt][2], av[mt][3]);
+        }
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
           uint32_t b0, b1;
           ldsm_x2(pt_addr + (8 * j + r8) * L::P_LD + (16 * kk + 8 * (mi & 1)) * 2, b0, b1);
-          mma_16816(oacc[j], a0, a1, a2, a3, b0, b1);
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) mma_16816(oacc[j][mt], av[mt][0], av[mt][1], av[mt][2], av[mt][3], b0, b1);
         }
       }
     }
@@ -300,13 +349,17 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
       const int n0 = 8 * j + 2 * tq;
-      if (n0 < g) {
-        po[n0 * D + ocol + grp] = oacc[j][0];
-        po[n0 * D + ocol + grp + 8] = oacc[j][2];
-      }
-      if (n0 + 1 < g) {
-        po[(n0 + 1) * D + ocol + grp] = oacc[j][1];
-        po[(n0 + 1) * D + ocol + grp + 8] = oacc[j][3];
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        const int col = ocol + 16 * mt + grp;
+        if (n0 < g) {
+          po[n0 * D + col] = oacc[j][mt][0];
+          po[n0 * D + col + 8] = oacc[j][mt][2];
+        }
+        if (n0 + 1 < g) {
+          po[(n0 + 1) * D + col] = oacc[j][mt][1];
+          po[(n0 + 1) * D + col + 8] = oacc[j][mt][3];
+        }
       }
     }
   } else {
@@ -315,10 +368,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
       const int n0 = 8 * j + 2 * tq;
-      red[(khalf * kDecMaxG + n0) * D + ocol + grp] = oacc[j][0];
-      red[(khalf * kDecMaxG + n0 + 1) * D + ocol + grp] = oacc[j][1];
-      red[(khalf * kDecMaxG + n0) * D + ocol + grp + 8] = oacc[j][2];
-      red[(khalf * kDecMaxG + n0 + 1) * D + ocol + grp + 8] = oacc[j][3];
+      red[(khalf * kDecMaxG + n0) * D + ocol + grp] = oacc[j][0][0];
+      red[(khalf * kDecMaxG + n0 + 1) * D + ocol + grp] = oacc[j][0][1];
+      red[(khalf * kDecMaxG + n0) * D + ocol + grp + 8] = oacc[j][0][2];
+      red[(khalf * kDecMaxG + n0 + 1) * D + ocol + grp + 8] = oacc[j][0][3];
     }
     __syncthreads();
     for (int idx = tid; idx < g * D; idx += kDecThreads) po[idx] = red[idx] + red[kDecMaxG * D + idx];

@@ -70,6 +70,8 @@ WORKLOADS = {
     "decode": Workload("decode", 8, 32, 32768, 128, "bf16", False, hkv=8, decode=True),
     # a training step at head dim 256 (forward + backward), 8192 tokens
     "train_d256": Workload("train_d256", 2, 8, 8192, 256, "bf16", True, backward=True),
+    # the decoding step of "decode" at head dim 256
+    "decode_d256": Workload("decode_d256", 8, 32, 32768, 256, "bf16", False, hkv=8, decode=True),
 }
 
 SINK_DELTAS = (0.0, 2.0, 4.0, 6.0, 7.0, 8.0, 10.0, 12.0)

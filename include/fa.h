@@ -15,8 +15,8 @@
  *    framework example); lse is a contiguous [B, H, N] float32 device array.
  *    LSE is the natural-log logsumexp of the scaled scores of each query row.
  *  - Sizes: B >= 1, H >= 1, N >= 1, d in {64, 128} (fa_fwd, fa_fwd_gqa, fa_bwd,
- *    fa_bwd_gqa and fa_bwd_noalloc also take d = 256, "FlashAttention (IT)",
- *    "FlashAttention-2"); B*H*N*d < 2^31.
+ *    fa_bwd_gqa, fa_bwd_noalloc and fa_decode also take d = 256, "FlashAttention
+ *    (IT)", "FlashAttention-2"); B*H*N*d < 2^31.
  *  - scale: the softmax scale (usually 1/sqrt(d)); finite and > 0.
  *  - causal != 0: query i attends to keys j <= i (square, top-left aligned);
  *    tiles that lie entirely in the future are skipped, never loaded.
@@ -137,8 +137,8 @@ int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const
  * reading the cache once: split over the key sequence with a log-sum-exp merge
  * of the chunks, K/V streamed by TMA, the per-chunk arithmetic on warp-level
  * tensor-core MMAs; the g = H / H_kv query heads of a key/value head are served
- * from one read of it (g <= 16).  Two launches on `stream` (split, combine). 
- * q, o: bf16 [B,H,d]; k, v: bf16 [B,H_kv,N,d]; lse: fp32 [B,H].
+ * from one read of it (g <= 16).  Two launches on `stream` (split, combine).
+ * q, o: bf16 [B,H,d]; k, v: bf16 [B,H_kv,N,d]; lse: fp32 [B,H]; d in {64, 128, 256}.
  * workspace: caller-owned, >= fa_decode_workspace_bytes(), 16-byte aligned. */
 size_t fa_decode_workspace_bytes(int B, int H, int H_kv, int N, int d);
 int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv, int N, int d,

@@ -70,6 +70,8 @@ def test_decode_workspace_size(lib):
         assert lib.fa_decode_workspace_bytes(*args) == expect(*args), args
     # the decode workload: 2 chunks of 128 tiles per key/value head
     assert expect(8, 32, 8, 32768, 128) == 2 * 8 * 32 * 130 * 4
+    for args in ((1, 8, 2, 1000, 256), (2, 16, 1, 4097, 256)):
+        assert lib.fa_decode_workspace_bytes(*args) == expect(*args) > 0
     assert lib.fa_decode_workspace_bytes(1, 6, 4, 100, 128) == 0   # H not a multiple of H_kv
     assert lib.fa_decode_workspace_bytes(1, 4, 4, 100, 96) == 0    # unsupported head dim
 

@@ -15,7 +15,10 @@ pytestmark = pytest.mark.gpu
 
 @pytest.mark.parametrize("B,H,Hkv,N,d", [(1, 8, 8, 1000, 128), (2, 32, 8, 4097, 128), (4, 16, 1, 333, 64),
                                          (1, 4, 4, 1, 64), (1, 16, 16, 70000, 128), (3, 12, 4, 65, 64),
-                                         (2, 24, 2, 5000, 128), (1, 8, 1, 129, 64)])
+                                         (2, 24, 2, 5000, 128), (1, 8, 1, 129, 64),
+                                         # head dim 256: the ring holds single K or V tiles
+                                         (1, 8, 2, 1000, 256), (2, 16, 1, 4097, 256), (1, 4, 4, 1, 256),
+                                         (1, 8, 8, 300, 256), (1, 16, 16, 40000, 256)])
 def test_decode_matches_oracle(B, H, Hkv, N, d):
     from exact_io_aware_85_b200 import fa
     rng_seed = 1300 + N + H
