@@ -43,9 +43,10 @@ def test_bwd_matches_finite_differences(causal):
         np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-8)
 
 
+@pytest.mark.parametrize("d", [16, 256])
 @pytest.mark.parametrize("causal", [False, True])
-def test_bwd_matches_torch_autograd_fp64(causal):
-    B, H, N, d = 2, 2, 33, 16
+def test_bwd_matches_torch_autograd_fp64(causal, d):
+    B, H, N = 2, 2, 33
     q, k, v, do = _inputs(B, H, N, d, seed=23)
     scale = 1.0 / math.sqrt(d)
     dq, dk, dv = oracle.attn_bwd(q, k, v, do, causal, scale)

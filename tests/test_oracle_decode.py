@@ -8,9 +8,10 @@ import oracle
 from exact_io_aware_85_b200 import synth
 
 
+@pytest.mark.parametrize("d", [16, 256])
 @pytest.mark.parametrize("Hq,Hkv", [(2, 2), (4, 1), (6, 3)])
-def test_decode_is_last_row_of_causal_attention(Hq, Hkv):
-    B, N, d = 2, 53, 16
+def test_decode_is_last_row_of_causal_attention(Hq, Hkv, d):
+    B, N = 2, 53
     x = synth.make_inputs(B, Hq, N, d, "f32", seed=Hq + 3 * Hkv)
     k, v = x["k"][:, :Hkv], x["v"][:, :Hkv]
     o_full, lse_full = oracle.attn_fwd_gqa(x["q"], k, v, True, 0.2)

@@ -18,7 +18,7 @@ def _rand(B, H, N, d, seed):
 
 
 @pytest.mark.parametrize("causal", [False, True])
-@pytest.mark.parametrize("shape", [(1, 2, 37, 16), (2, 1, 64, 32), (1, 1, 1, 8)])
+@pytest.mark.parametrize("shape", [(1, 2, 37, 16), (2, 1, 64, 32), (1, 1, 1, 8), (1, 2, 37, 256)])
 def test_fwd_matches_torch_sdpa_fp64(shape, causal):
     q, k, v = _rand(*shape, seed=3)
     scale = 1.0 / math.sqrt(shape[-1])

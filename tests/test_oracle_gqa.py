@@ -28,9 +28,10 @@ def test_gqa_forward_is_mha_with_shared_heads(Hq, Hkv, causal):
     np.testing.assert_allclose(l, l_ref, atol=1e-13)
 
 
+@pytest.mark.parametrize("d", [8, 256])
 @pytest.mark.parametrize("Hq,Hkv", [(4, 2), (3, 1)])
-def test_gqa_backward_matches_torch_autograd(Hq, Hkv):
-    B, N, d = 1, 23, 8
+def test_gqa_backward_matches_torch_autograd(Hq, Hkv, d):
+    B, N = 1, 23
     x = synth.make_inputs(B, Hq, N, d, "f32", seed=7, with_grad=True)
     q = x["q"].astype(np.float64)
     k = x["k"][:, :Hkv].astype(np.float64)
