@@ -729,13 +729,15 @@ __global__ void __launch_bounds__(448, 1)
         for (int k = 0; k < 4; ++k)
           mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + 64 * b + (k >> 1) * 32 + (k & 1) * 8,
                  make_sdesc_sw128(qa + k * 2048, C::Q_BOX, 1024), id_g, (u > 0 || k > 0) ? 1u : 0u);
+        // dK was the stage's last reader (the gradient warps are done with its
+        // LSE and D): release it before dQ^T, which reads only K_j and dS^T
+        mma_commit(bar_ld_empty + su);
         // dQ_i^T = K_j^T dS^T   (M = 128 columns, N = 64 queries, K = 128 keys), over S^T(u)
 #pragma unroll
         for (int k = 0; k < 8; ++k)
           mma_ss(tmem + C::COL_S + 64 * b, make_sdesc_sw128(kh + k * 2048, C::KV_BOX, 1024),
                  make_sdesc_sw128(dsa + k * 2048, C::KV_BOX, 1024), id_q, k > 0 ? 1u : 0u);
         mma_commit(bar_dq_full + b);
-        mma_commit(bar_ld_empty + su);
         mma_commit(bar_pds_free + b);
         return true;
       };
