@@ -96,3 +96,25 @@ def test_argument_errors_need_no_gpu(lib):
     ws_small = 10
     assert lib.fa_bwd(*([good] * 9), 1, 1, 64, 128, 1, 0.1, good, ws_small, None) == 1
     assert lib.fa_bwd(*([good] * 9), 1, 1, 64, 128, 1, 0.1, vp((1 << 20) + 16), 1 << 30, None) == 3
+
+
+def test_head_dim_256_is_admitted_where_declared(lib):
+    """d = 256 passes the argument checks of the entry points that declare it
+    (their next check, a short workspace or a misaligned pointer, is the one that
+    fails) and is refused with FA_ERR_UNSUPPORTED by those that do not."""
+    vp, ci, cf, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    good = vp(1 << 20)
+    bad = vp((1 << 20) + 8)
+    lib.fa_bwd.argtypes = [vp] * 9 + [ci] * 5 + [cf, vp, sz, vp]
+    assert lib.fa_bwd(*([good] * 9), 1, 1, 64, 256, 1, 0.1, good, 10, None) == 1          # workspace too small
+    assert lib.fa_bwd(*([good] * 9), 1, 1, 64, 96, 1, 0.1, good, 1 << 30, None) == 2      # unsupported
+    lib.fa_bwd_gqa.argtypes = [vp] * 9 + [ci] * 6 + [cf, vp, sz, vp]
+    assert lib.fa_bwd_gqa(*([good] * 9), 1, 4, 2, 64, 256, 1, 0.1, good, 10, None) == 1
+    lib.fa_bwd_noalloc.argtypes = [vp] * 9 + [ci] * 5 + [cf, vp]
+    assert lib.fa_bwd_noalloc(*([good] * 4), bad, *([good] * 4), 1, 1, 64, 256, 1, 0.1, None) == 3  # dO misaligned
+    lib.fa_decode.argtypes = [vp] * 5 + [ci] * 5 + [cf, vp, sz, vp]
+    assert lib.fa_decode(good, good, good, good, good, 1, 4, 1, 64, 256, 0.1, good, 10, None) == 1
+    assert lib.fa_decode(good, good, good, good, good, 1, 4, 1, 64, 96, 0.1, good, 1 << 30, None) == 2
+    assert lib.fa_decode(good, good, good, good, good, 1, 32, 1, 64, 256, 0.1, good, 1 << 30, None) == 2  # g > 16
+    lib.fa_fwd_fp8.argtypes = [vp] * 3 + [vp] * 3 + [vp, vp] + [ci] * 5 + [cf, cf, ci, vp]
+    assert lib.fa_fwd_fp8(*([good] * 8), 1, 1, 64, 256, 1, 0.1, 256.0, 0, None) == 2      # FP8 takes d = 128
