@@ -438,7 +438,7 @@ __global__ void __launch_bounds__(448, 1)
 }
 
 // ---------------------------------------------------------------------------
-// bwd_main, pipelined variant for d = 128 (64-query steps)
+// bwd_main, pipelined variant for d = 128 and 256 (64-query steps)
 // ---------------------------------------------------------------------------
 // Tensor memory at d = 128 cannot hold a second 128-query S^T tile, so this
 // variant walks the query tiles 64 at a time and double-buffers everything:
@@ -456,8 +456,8 @@ __global__ void __launch_bounds__(448, 1)
 // dQ^T = K^T dS^T (M = d lanes, N = 64 queries), so the drain warps (thread =
 // head dimension) add into the fp32 accumulator with fully coalesced reductions.
 //
-// Head dimension 256 ("FlashAttention (IT)", section "FlashAttention-2": head
-// dimensions up to 256) does not fit this tensor-memory budget whole: dV and dK
+// Head dimension 256 ("FlashAttention (IT)", section "FlashAttention-2 (2023)":
+// heads up to 256 wide) does not fit this tensor-memory budget whole: dV and dK
 // of a 128-key tile alone would take all 512 columns.  Each CTA therefore owns
 // one 128-wide slice of the head dimension (blockIdx.y): S^T and dP^T contract
 // over all 256 columns (recomputed by both CTAs of a key tile), while dV, dK and

@@ -1,5 +1,5 @@
 // fwd256.cuh — exact attention forward for head dim 256 ("FlashAttention (IT)",
-// "FlashAttention-2": head dimension up to 256), same algorithm as fwd.cuh.
+// "FlashAttention-2 (2023)": head dimension up to 256), same algorithm as fwd.cuh.
 //
 // At d = 256 the fp32 output tile of 128 query rows alone takes 256 of the 512
 // tensor-memory columns, so the two-Q-tile ping-pong of fwd.cuh does not fit.

@@ -16,7 +16,7 @@
  *    LSE is the natural-log logsumexp of the scaled scores of each query row.
  *  - Sizes: B >= 1, H >= 1, N >= 1, d in {64, 128} (fa_fwd, fa_fwd_gqa, fa_bwd,
  *    fa_bwd_gqa, fa_bwd_noalloc and fa_decode also take d = 256, "FlashAttention
- *    (IT)", "FlashAttention-2"); B*H*N*d < 2^31.
+ *    (IT)", "FlashAttention-2 (2023)"); B*H*N*d < 2^31.
  *  - scale: the softmax scale (usually 1/sqrt(d)); finite and > 0.
  *  - causal != 0: query i attends to keys j <= i (square, top-left aligned);
  *    tiles that lie entirely in the future are skipped, never loaded.
@@ -116,7 +116,7 @@ int fa_fwd_fp8p(const void* q, const void* k, const void* v, void* o, float* lse
 
 /* Grouped-query / multi-query attention ("FlashAttention for Scalable Vector
  * Architectures", "Metodologia": a key/value head shared by several query heads;
- * "FlashAttention (IT)", "FlashAttention-2": Multi-Query Attention).
+ * "FlashAttention (IT)", "FlashAttention-2 (2023)": Multi-Query Attention).
  * q, o: [B,H,N,d]; k, v: [B,H_kv,N,d] with H a multiple of H_kv; query head h
  * uses key/value head h / (H / H_kv).  H_kv = 1 is multi-query attention,
  * H_kv = H is fa_fwd.  lse: [B,H,N].  Other conventions as fa_fwd. */
