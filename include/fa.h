@@ -29,7 +29,12 @@
  *    returns FA_ERR_CUDA (fa_last_cuda_error() gives the cudaError_t).  Device
  *    pipelines that stall past a bound record FA_ERR_TIMEOUT in a device status
  *    word that fa_check_status() reads after the caller's work has finished.
- *  - Thread safety: entry points may be called concurrently from host threads.
+ *  - Thread safety: entry points may be called concurrently from host threads,
+ *    with these shared parts: fa_last_cuda_error() is per host thread; the
+ *    timeout status word is per device and shared by every caller in the
+ *    process, so fa_check_status() reports (and clears) a timeout raised by any
+ *    thread's kernels on the current device; fa_bwd_noalloc calls share one
+ *    scratch array per device and must not overlap on the GPU.
  */
 #ifndef FA_H_
 #define FA_H_
