@@ -142,6 +142,11 @@ def fa_check_status() -> int:
     return int(lib.fa_check_status())
 
 
+def fa_last_cuda_error() -> int:
+    """The cudaError_t of this host thread's last failed CUDA call inside the library."""
+    return int(lib.fa_last_cuda_error())
+
+
 def fa_watchdog_selftest(limit_us: int, stream=None) -> None:
     _check(lib.fa_watchdog_selftest(int(limit_us), _stream(stream)), "fa_watchdog_selftest")
 

@@ -1,8 +1,12 @@
 """The Python binding checks every tensor argument (CUDA, contiguous, dtype,
 shape, one device) before it calls into the library; on this CPU host the
 checks fire on CPU tensors, so no CUDA call is made."""
+import os
+
 import pytest
 import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def _fa():
@@ -39,3 +43,14 @@ def test_need_checks_dtype_and_shape_in_order():
     fa._need("x", a=(None, torch.float32, None))
     with pytest.raises(fa.FAError):
         fa._need("x", a=(None, torch.float32, (4,)))
+
+
+def test_every_entry_point_has_a_binding_of_the_same_name():
+    """The Python layer mirrors the C ABI name for name (argument marshalling only)."""
+    import re
+
+    from exact_io_aware_85_b200 import fa
+    header = open(os.path.join(ROOT, "include", "fa.h")).read()
+    declared = set(re.findall(r"^\s*(?:int|size_t|const char\*)\s+(fa_\w+)\(", header, re.M))
+    assert len(declared) >= 16
+    assert sorted(n for n in declared if not callable(getattr(fa, n, None))) == []
