@@ -130,3 +130,65 @@ def test_mse_orderings_from_the_page(sweep):
     for delta in (7.0, 10.0, 12.0):
         assert mse[(delta, 448.0, 0)] > mse[(delta, 256.0, 0)]  # S=256 never worse than 448
         assert abs(mse[(delta, 256.0, 1)] / mse[(delta, 256.0, 0)] - 1.0) < 0.1  # reverse ~ forward at S=256
+
+
+def _ln2_ladder(descending: bool):
+    """Logits on a ln 2 ladder: key tile t of 4 keys holds a maximum 2 t ln 2 (or
+    2 (T-1-t) ln 2 when descending) and keys 0, 1, 5, 9 ln 2 below it, so
+    within a row every score sits a whole number n <= 17 of ln 2 below any
+    running maximum it can meet, in either key order and at any causal cut.
+    Then S p = 256 * 2^-n is an E4M3 value (2^-9 is the smallest), the cast is
+    exact while the maximum keeps moving from tile to tile, and the emulation
+    must reproduce exact attention, rescaling of the accumulator included."""
+    T, steps = 5, (0, 1, 5, 9)
+    ln2 = math.log(2.0)
+    logits = []
+    for t in range(T):
+        top = 2 * (T - 1 - t if descending else t)
+        logits += [(top - n) * ln2 for n in steps]
+    N = len(logits)
+    q = np.zeros((1, 1, N, 3))
+    q[..., 0] = 1.0
+    k = np.zeros((1, 1, N, 3))
+    k[0, 0, :, 0] = logits
+    v = np.random.default_rng(3).standard_normal((1, 1, N, 3))
+    return q, k, v
+
+
+@pytest.mark.parametrize("descending", [False, True])
+@pytest.mark.parametrize("order", [0, 1])
+@pytest.mark.parametrize("causal", [False, True])
+def test_grid_exact_p_with_moving_max_gives_exact_attention(descending, order, causal):
+    q, k, v = _ln2_ladder(descending)
+    o_ref, lse_ref = oracle.attn_fwd(q, k, v, causal, 1.0)
+    o, lse, counts = oracle.attn_fwd_fp8p(q, k, v, causal, 1.0, 256.0, order, Bc=4, n_sink=0)
+    np.testing.assert_allclose(o, o_ref, atol=1e-12, rtol=0)
+    np.testing.assert_allclose(lse, lse_ref, atol=1e-12, rtol=0)
+    assert counts[2] == 0
+
+
+def test_flushed_p_leave_the_numerator_but_not_the_sum():
+    """Scores 19 and 21 ln 2 below their tile's maximum (forward order, maxima
+    growing tile by tile): S p = 2^-11 and 2^-13 round to zero, so those keys
+    drop out of the numerator of O while their unquantised p stays in the
+    denominator l; every other S p is on the E4M3 grid.  (The 2^-10 tie itself
+    cannot be reached through exp in fp64, which misses 2^-18 by an ulp; the
+    E4M3 tests pin it.)  The expected O is written from that definition."""
+    ln2 = math.log(2.0)
+    shifts = (0, 3, 19, 21)
+    logits = [(2 * t - n) * ln2 for t in range(4) for n in shifts]
+    N = len(logits)
+    q = np.zeros((1, 1, N, 2))
+    q[..., 0] = 1.0
+    k = np.zeros((1, 1, N, 2))
+    k[0, 0, :, 0] = logits
+    v = np.random.default_rng(4).standard_normal((1, 1, N, 2))
+    s = np.array(logits)
+    e = np.exp(s - s.max())
+    kept = np.array([n <= 17 for _ in range(4) for n in shifts])
+    o_want = (e[kept, None] * v[0, 0][kept]).sum(axis=0) / e.sum()
+    o, lse, counts = oracle.attn_fwd_fp8p(q, k, v, False, 1.0, 256.0, 0, Bc=4, n_sink=0)
+    for i in range(N):
+        np.testing.assert_allclose(o[0, 0, i], o_want, atol=1e-12, rtol=0)
+    assert counts[2] == N * 8 and counts[3] == N * N  # 2 flushed keys per tile, every row
+    np.testing.assert_allclose(lse[0, 0], np.log(np.exp(s).sum()), atol=1e-12)
