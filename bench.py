@@ -34,9 +34,9 @@ sys.path.insert(0, ROOT)
 from exact_io_aware_85_b200 import synth  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM traffic per launch of the dominant kernel, from the ncu captures summarised
-# in profiles/ (fa_fwd_prefill.md, fa_decode.md); reported only while the kernel
-# sources still hash to the values they were measured with.
+# DRAM traffic per launch of the dominant kernel, from one-pass ncu captures of
+# that kernel (dram__bytes_read.sum + dram__bytes_write.sum); reported only while
+# the kernel sources still hash to the values they were measured with.
 TRAFFIC = {
     "prefill": {"bytes": 806519296 + 252521472, "src": ("fwd.cuh", "sm100.cuh"),
                 "sha1": "032a7705e1c46488fe7ced39baa01ab1630e52bc"},
@@ -164,6 +164,29 @@ def device_inputs(w: synth.Workload, seed: int):
     return q, k, v
 
 
+def measure_fp8_peak(n: int = 8192, reps: int = 10):
+    """Dense E4M3 GEMM throughput of this GPU: torch._scaled_mm (cuBLASLt) on
+    n x n x n E4M3 operands with bf16 output, the best of `reps` CUDA-event
+    timed launches after warm-up, the way the bf16 peak is measured (a burst)."""
+    g = torch.Generator(device="cuda")
+    g.manual_seed(12345)
+    a = torch.randn((n, n), generator=g, device="cuda").to(torch.float8_e4m3fn)
+    b = torch.randn((n, n), generator=g, device="cuda").to(torch.float8_e4m3fn).t()  # column-major operand
+    one = torch.ones((), dtype=torch.float32, device="cuda")
+    for _ in range(3):
+        torch._scaled_mm(a, b, one, one, out_dtype=torch.bfloat16)
+    best = float("inf")
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        torch._scaled_mm(a, b, one, one, out_dtype=torch.bfloat16)
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    del a, b
+    return 2.0 * n ** 3 / (best * 1e-3) / 1e12
+
+
 def cpu_baseline(w: synth.Workload, target_s: float = 12.0):
     """The fp64 oracle on the host cores over a bounded sample of query rows of
     the same workload; TFLOP/s of useful attention work."""
@@ -223,6 +246,10 @@ METRIC = "attention fwd/bwd TFLOP/s at 1 B200 and % of dense BF16/FP8 tensor pea
 
 def config_of(w, ws):
     what = ("forward + backward (dQ, dK, dV from the saved LSE)" if w.backward else
+            "bf16 forward without the cast (the sink workload's reference cost), sink Delta=8"
+            if w.sink and w.variant == "bf16" else
+            "FP8 P-cast forward, S=256, forward key order, sink Delta=8, no flush counting"
+            if w.sink and w.variant == "nostats" else
             "FP8 P-cast forward, S=256, forward key order, sink Delta=8" if w.sink else
             "E4M3 forward (Hadamard-rotated block-quantised Q/K, per-head V, P-cast S=256)" if w.dtype == "fp8"
             else "forward (O + LSE)")
@@ -274,10 +301,14 @@ def main():
         k[..., :4, 0] = 8.0 * math.sqrt(w.d)
         k[..., 4:, 0] = 0.0
         q[..., 0] = 1.0
-        stats = torch.zeros(4, dtype=torch.int64, device="cuda")
+        stats = torch.zeros(4, dtype=torch.int64, device="cuda") if not w.variant else None
 
-        def run():
-            fa.fa_fwd_fp8p(q, k, v, o, lse, w.causal, w.scale, 256.0, 0, stats, 4)
+        if w.variant == "bf16":
+            def run():
+                fa.fa_fwd(q, k, v, o, lse, w.causal, w.scale)
+        else:
+            def run():
+                fa.fa_fwd_fp8p(q, k, v, o, lse, w.causal, w.scale, 256.0, 0, stats, 4)
     elif w.dtype == "fp8":
         # E4M3 operands prepared once (quantisation with the random-sign Hadamard
         # rotation, outside the timed step); the step is the FP8 attention kernel
@@ -400,10 +431,12 @@ def main():
 
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     peak_note = f"{peak_src} bf16 burst (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback 1590 TFLOP/s"
+    fp8_peak = None
     if w.dtype == "fp8":
-        # no measured FP8 peak is available: the measured bf16 peak x the nominal 2x FP8 ratio
-        peak *= 2.0
-        peak_note = f"{peak_src} bf16 burst x 2 (nominal FP8/BF16 ratio)"
+        # the E4M3 contraction is held against an E4M3 GEMM measured here, now
+        fp8_peak = measure_fp8_peak()
+        peak = fp8_peak
+        peak_note = "E4M3 GEMM burst measured in this run (torch._scaled_mm 8192^3, best of 10)"
     bound, unit, peak_val = "tensor", "TFLOP/s", peak
     if w.decode:
         # bound by reading the key/value cache: roofline in bytes against measured HBM
@@ -414,7 +447,8 @@ def main():
         kernel_name = "training step: %s + fa_bwd (pre, main, post)" % (
             "fa_fwd256_kernel" if w.d == 256 else "fa_fwd_kernel<bf16,%d>" % w.d)
     elif w.sink:
-        kernel_name = "fa_fwd_kernel<bf16,%d,FP8P>" % w.d
+        kernel_name = ("fa_fwd_kernel<bf16,%d> (no cast)" % w.d if w.variant == "bf16" else
+                       "fa_fwd_kernel<bf16,%d,FP8P%s>" % (w.d, "" if w.variant else ",COUNT"))
     elif w.dtype == "fp8":
         kernel_name = "fa_fwd_kernel<e4m3,%d> (kind::f8f6f4)" % w.d
     elif w.decode:
@@ -426,6 +460,29 @@ def main():
     else:
         kernel_name = "fa_fwd_kernel<%s,%d>" % ("bf16" if w.dtype == "bf16" else "f32/tf32", w.d)
     achieved = flops / (step_ms_local * 1e-3) / 1e12
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    hbm = None
+    if w.name == "tiny":
+        # short sequence: the algorithmic bytes (Q, K, V read, O and LSE written once) over the launch time
+        nbytes = 4 * q.numel() * q.element_size() + lse.numel() * 4
+        hbm = {"what": "fa_fwd_f32 launch", "algorithmic_bytes": nbytes,
+               "achieved_gbs": nbytes / (step_ms_local * 1e-3) / 1e9,
+               "frac_of_measured": nbytes / (step_ms_local * 1e-3) / 1e9 / hbm_peak}
+    elif w.backward:
+        # the backward alone (pre, main, post), timed after the step: Q, K, V, O, dO read and dQ, dK, dV
+        # written once in bf16, LSE read, plus the fp32 dQ accumulator zeroed once and read once
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        for _ in range(args.steps):
+            fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, w.causal, w.scale, ws_buf)
+        b1.record(stream)
+        torch.cuda.synchronize()
+        bwd_ms = b0.elapsed_time(b1) / args.steps
+        nbytes = 8 * q.numel() * 2 + lse.numel() * 4 + 2 * q.numel() * 4
+        hbm = {"what": "fa_bwd (pre + main + post) alone", "ms": bwd_ms, "algorithmic_bytes": nbytes,
+               "achieved_gbs": nbytes / (bwd_ms * 1e-3) / 1e9,
+               "frac_of_measured": nbytes / (bwd_ms * 1e-3) / 1e9 / hbm_peak,
+               "tflops": w.bwd_flops() / (bwd_ms * 1e-3) / 1e12}
     if w.decode:
         achieved_bytes = (sum(t.numel() * t.element_size() for t in (q, k, v, o)) + lse.numel() * 4) / (
             step_ms_local * 1e-3) / 1e9
@@ -456,6 +513,10 @@ def main():
         }
         if w.dtype == "fp8":
             line["fp8_quantize_ms"] = quant_ms
+            line["fp8_peak_tflops"] = fp8_peak
+            line["pct_of_peak"]["measured_e4m3_burst"] = achieved / fp8_peak
+        if hbm is not None:
+            line["hbm"] = hbm
         if ws == 1 and not args.no_cpu_baseline:
             cb = cpu_baseline(w)
             cb.pop("seconds", None)

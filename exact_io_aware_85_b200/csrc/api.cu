@@ -81,19 +81,34 @@ int encode_qkv_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int
   return FA_OK;
 }
 
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// Size limits, set by what the launches can express rather than by memory:
+// N <= 2^30 (row indices and 256-row block offsets stay int), B*H < 2^31 and
+// fewer than 2^31 CTAs in the largest grid (B*H x 128-row blocks, gridDim.x),
+// and B*H*N*d < 2^40 elements (the one-thread-per-8-elements grids of the
+// backward's pre and post passes).  Element offsets are 64-bit everywhere.
+bool sizes_fit(int B, int H, int N, int d) {
+  if (N > (1 << 30)) return false;
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH >= (1ll << 31)) return false;
+  if (BH * ((static_cast<long long>(N) + 127) / 128) >= (1ll << 31)) return false;
+  return BH * N * d < (1ll << 40);
+}
+
 int check_common(const void* q, const void* k, const void* v, const void* o, const void* lse, int B, int H, int N,
                  int d, float scale, bool allow256 = false) {
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
   if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128 && !(allow256 && d == 256)) return FA_ERR_UNSUPPORTED;
-  const long long total = static_cast<long long>(B) * H * N * d;
-  if (total >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGNMENT;
+  if (!sizes_fit(B, H, N, d)) return FA_ERR_UNSUPPORTED;
+  // lse is written one fp32 scalar at a time
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse)) return FA_ERR_ALIGNMENT;
   return FA_OK;
 }
 
-template <typename T, int D, bool FP8P>
+template <typename T, int D, bool FP8P, bool COUNT = false>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int causal,
                float scale, float S, int kv_order, unsigned long long* stats, int n_sink, cudaStream_t stream,
                const float* sq = nullptr, const float* sk = nullptr, const float* sv = nullptr, int Hkv = 0) {
@@ -128,7 +143,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   a.sv = sv;
   a.nqb = (N + 127) / 128;
   a.group = H / Hkv;
-  auto kern = fa::fa_fwd_kernel<T, D, FP8P>;
+  auto kern = fa::fa_fwd_kernel<T, D, FP8P, COUNT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_fail(e);
   const long long grid = static_cast<long long>(a.nblk) * BH;
@@ -226,27 +241,66 @@ int launch_bwd_d(int d, const void* q, const void* k, const void* v, const void*
 // kernel (on the host it only stands for the symbol); each device's address of
 // it is looked up once with cudaGetSymbolAddress and cached.
 // ---------------------------------------------------------------------------
-constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB, held by every GPU that loads the library
+constexpr size_t kNoAllocScratchBytes = FA_BWD_NOALLOC_MAX_BYTES;  // 32 MiB, held by every GPU that loads the library
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
+// per device: the address of the array and the id of the CUDA context it was
+// looked up in (a reset device gets a new context, whose id is new for the life
+// of the process, and the address is looked up again)
 void* g_noalloc_ptr[kMaxDevices] = {};
+unsigned long long g_noalloc_ctx[kMaxDevices] = {};
+
+using PFN_ctx_get_current = CUresult (*)(CUcontext*);
+using PFN_ctx_get_id = CUresult (*)(CUcontext, unsigned long long*);
+
+// Id of the context current on this thread, 0 if there is none yet (the
+// runtime makes one current at its first call that needs it) or the driver
+// cannot tell; with 0 the address is looked up again on every call.
+unsigned long long current_context_id() {
+  static PFN_ctx_get_current get_cur = nullptr;
+  static PFN_ctx_get_id get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<PFN_ctx_get_current>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_ctx_get_id>(p);
+  });
+  if (!get_cur || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_cur(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 }  // namespace
 
 static __device__ __align__(256) unsigned char g_bwd_scratch[kNoAllocScratchBytes];
+static_assert(sizeof(g_bwd_scratch) == FA_BWD_NOALLOC_MAX_BYTES, "scratch array size is the header's limit");
 
 namespace {
+// The device address of the scratch array in the current context.  On the host
+// the array's name only stands for the symbol; the address is looked up with
+// cudaGetSymbolAddress once per device and context, with that device current.
 int noalloc_scratch_for_current_device(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
   if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  if (g_noalloc_ptr[dev] == nullptr || ctx == 0 || g_noalloc_ctx[dev] != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_bwd_scratch);
     if (e != cudaSuccess) return cuda_fail(e);
     g_noalloc_ptr[dev] = p;
+    g_noalloc_ctx[dev] = ctx;
   }
   *out = g_noalloc_ptr[dev];
   return FA_OK;
@@ -339,9 +393,16 @@ int fa_fwd_fp8p(const void* q, const void* k, const void* v, void* o, float* lse
   if (n_sink < 0) return FA_ERR_INVALID_ARG;
   if (stats && (reinterpret_cast<uintptr_t>(stats) & 7u)) return FA_ERR_ALIGNMENT;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the flush counting is a separate instantiation: without stats the kernel carries none of it
   if (d == 64)
-    return launch_fwd<__nv_bfloat16, 64, true>(q, k, v, o, lse, B, H, N, causal, scale, S, kv_order, stats, n_sink, s);
-  return launch_fwd<__nv_bfloat16, 128, true>(q, k, v, o, lse, B, H, N, causal, scale, S, kv_order, stats, n_sink, s);
+    return stats ? launch_fwd<__nv_bfloat16, 64, true, true>(q, k, v, o, lse, B, H, N, causal, scale, S, kv_order,
+                                                             stats, n_sink, s)
+                 : launch_fwd<__nv_bfloat16, 64, true>(q, k, v, o, lse, B, H, N, causal, scale, S, kv_order, nullptr,
+                                                       n_sink, s);
+  return stats ? launch_fwd<__nv_bfloat16, 128, true, true>(q, k, v, o, lse, B, H, N, causal, scale, S, kv_order,
+                                                            stats, n_sink, s)
+               : launch_fwd<__nv_bfloat16, 128, true>(q, k, v, o, lse, B, H, N, causal, scale, S, kv_order, nullptr,
+                                                      n_sink, s);
 }
 
 int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv, int N, int d,
@@ -388,7 +449,8 @@ int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, 
   if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
   const int g = H / H_kv;
   if (g > fa::kDecMaxG) return FA_ERR_UNSUPPORTED;
-  if (static_cast<long long>(B) * H_kv * N * d >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
+  if (!sizes_fit(B, H, N, d)) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H_kv > 65535) return FA_ERR_UNSUPPORTED;  // key/value heads are gridDim.y
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
       (reinterpret_cast<uintptr_t>(workspace) & 15u))
     return FA_ERR_ALIGNMENT;
@@ -436,7 +498,8 @@ int fa_fp8_quantize(const void* q, const void* k, const void* v, const float* si
   if (!q || !k || !v || !q8 || !k8 || !v8 || !sq || !sk || !sv) return FA_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
-  if (static_cast<long long>(B) * H * N * d >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
+  if (!sizes_fit(B, H, N, d)) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H > 65535) return FA_ERR_UNSUPPORTED;  // heads are gridDim.y of the Q/K pass
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q8) || !aligned16(k8) || !aligned16(v8))
     return FA_ERR_ALIGNMENT;
   if ((reinterpret_cast<uintptr_t>(sq) | reinterpret_cast<uintptr_t>(sk) | reinterpret_cast<uintptr_t>(sv) |
@@ -542,15 +605,16 @@ const char* fa_status_string(int status) {
 
 int fa_last_cuda_error(void) { return t_last_cuda_error; }
 
-int fa_check_status(void) {
-  cudaError_t e = cudaDeviceSynchronize();
-  if (e != cudaSuccess) return cuda_fail(e);
+int fa_check_status(void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
   int v = 0;
-  e = cudaMemcpyFromSymbol(&v, fa::g_fa_status, sizeof(int));
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&v, fa::g_fa_status, sizeof(int), 0, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e);
   if (v != 0) {
-    const int zero = 0;
-    e = cudaMemcpyToSymbol(fa::g_fa_status, &zero, sizeof(int));
+    static const int zero = 0;
+    e = cudaMemcpyToSymbolAsync(fa::g_fa_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_fail(e);
   }
   return v & 0xFF;

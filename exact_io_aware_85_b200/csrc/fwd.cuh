@@ -95,6 +95,16 @@ struct FwdCfg {
   // takes ~151 cycles per 16-deep step against ~108 from shared memory (at
   // N = 128, d = 128, tensor memory is the faster, ~73).
   static constexpr bool PV_SS = (EB == 2) && (D == 64) && !FP8P;
+  // Exponentials on the FMA pipe (exp2_fma2): this many of every 8 key pairs of
+  // a bf16 tile, the rest on the MUFU.  At d = 64 the MUFU is the busiest pipe
+  // (one exp per 128 FLOP of MMA against one per 256 at d = 128).
+#ifndef FA_EXP_POLY_D64
+#define FA_EXP_POLY_D64 0
+#endif
+#ifndef FA_EXP_POLY_D128
+#define FA_EXP_POLY_D128 0
+#endif
+  static constexpr int EXP_POLY = (EB == 2 && !FP8P) ? (D == 64 ? FA_EXP_POLY_D64 : FA_EXP_POLY_D128) : 0;
   static constexpr int P_BYTES = 128 * 128 * 2;  // one 128 x 128 bf16 P tile: two 64-key boxes
   static constexpr int OFF_P = OFF_V + NSTAGE * TILE_BYTES;
   static constexpr int SMEM_BYTES = OFF_P + (PV_SS ? 2 * P_BYTES : 0) + 1024;  // + alignment slack
@@ -104,7 +114,9 @@ struct FwdCfg {
   static_assert(COL_O1 + D <= 512, "tensor memory budget");
 };
 
-template <typename T, int D, bool FP8P>
+// FP8P: P is cast to E4M3 before PV (bf16 operands); COUNT: FP8P that also
+// counts the P' values that flushed to zero.
+template <typename T, int D, bool FP8P, bool COUNT = false>
 __global__ void __launch_bounds__(320, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
@@ -362,8 +374,12 @@ __global__ void __launch_bounds__(320, 1)
     // scale*log2(e) * sq[query block] * sk[key block j]
     const float c_base = C::EB == 1 ? a.scale_log2 * a.sq[static_cast<size_t>(bh) * a.nqb + qt] : a.scale_log2;
     const int bh_k = bh_kv;  // key-side scales are per key/value head
+    // With a P-cast (FP8P or E4M3 operands) the exponent carries log2(S): the
+    // exps give q = S p directly, l sums q, and the epilogue divides by it.
+    constexpr bool kCast = FP8P || C::EB == 1;
+    const float lg2S = kCast ? log2f(a.p_scale) : 0.f;
     float m_run = -INFINITY, l_run = 0.f;
-    uint32_t fl_sink = 0, fl_non = 0;
+    uint32_t nf_sink = 0, nf_non = 0;  // COUNT: P' that did not flush, per key class
     int cnt = 0;
     bool ok = true;
     if (kv_end > 0) {
@@ -419,12 +435,28 @@ __global__ void __launch_bounds__(320, 1)
         const bool rescale = cnt > 0 && __any_sync(0xffffffffu, m_new != m_run);
         l_run *= alpha;
         m_run = m_new;
-        const float neg_m = -m_run;
+        const float neg_m = lg2S - m_run;
         // 4 independent pairs of partial row sums (packed fp32x2 adds)
         float2 rs4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         const float2 c2 = make_float2(c, c), nm2 = make_float2(neg_m, neg_m);
-        // FP8 flush counting: tiles with no masked key and no sink key need no per-key test
-        const bool plain_tile = !masked_tile && kbase >= a.n_sink;
+        // COUNT, tiles that hold sink keys: the P' of keys < n_sink that did not
+        // flush, counted apart before the main pass (the same fma, ex2 and cast
+        // as there, so the same values); the main pass counts every key.
+        uint32_t nf_part = 0;
+        if constexpr (COUNT) {
+          if (kbase < a.n_sink && row < N) {
+#pragma unroll
+            for (int cc = 0; cc < 128; ++cc) {
+              if (kbase + cc < a.n_sink) {
+                const float qv = ex2_approx(fmaf(sv[cc], c, neg_m));
+                uint16_t e8;
+                asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(e8) : "f"(0.f), "f"(qv));
+                nf_part += (e8 & 0xFFu) ? 1u : 0u;
+              }
+            }
+          }
+        }
+        uint32_t nf_tile = 0;
         if constexpr (C::EB == 1) {
           // P' = E4M3(S p), four codes per 32-bit TMEM column (the PV MMA's A operand)
           uint32_t pk[32];
@@ -432,11 +464,9 @@ __global__ void __launch_bounds__(320, 1)
           for (int e = 0; e < 32; ++e) {
             const float2 x01 = ffma2(make_float2(sv[4 * e], sv[4 * e + 1]), c2, nm2);
             const float2 x23 = ffma2(make_float2(sv[4 * e + 2], sv[4 * e + 3]), c2, nm2);
-            const float2 p01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
-            const float2 p23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
-            rs4[e & 3] = fadd2(rs4[e & 3], fadd2(p01, p23));
-            const float2 s01 = fmul2(p01, make_float2(a.p_scale, a.p_scale));
-            const float2 s23 = fmul2(p23, make_float2(a.p_scale, a.p_scale));
+            const float2 s01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));  // S p
+            const float2 s23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
+            rs4[e & 3] = fadd2(rs4[e & 3], fadd2(s01, s23));
             uint16_t lo, hi;
             asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(s01.y), "f"(s01.x));
             asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(s23.y), "f"(s23.x));
@@ -451,37 +481,29 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
           for (int h = 0; h < 64 / PC; ++h) {
             uint32_t pk[PC];
-            // FP8 P-cast flush counting: per pair, bit 0 / bit 16 of nz = "this P' is
-            // not zero".  Tiles without masked or sink keys only add up the flags (two
-            // 16-bit counters in one word), settled once per chunk.
-            uint32_t nzacc = 0;
-            const bool count_each = FP8P && a.stats != nullptr && !plain_tile && row < N;
+            uint32_t nz2 = 0;  // COUNT: f16x2 counter of non-zero P' in this chunk
 #pragma unroll
             for (int e = 0; e < PC; ++e) {
               const float2 x = ffma2(make_float2(sv[h * 2 * PC + 2 * e], sv[h * 2 * PC + 2 * e + 1]), c2, nm2);
-              const float p0 = ex2_approx(x.x);
-              const float p1 = ex2_approx(x.y);
+              float p0, p1;  // S p with FP8P, p otherwise
+              if ((e & 7) < C::EXP_POLY) {
+                const float2 pp = exp2_fma2(x);
+                p0 = pp.x;
+                p1 = pp.y;
+              } else {
+                p0 = ex2_approx(x.x);
+                p1 = ex2_approx(x.y);
+              }
               rs4[e & 3] = fadd2(rs4[e & 3], make_float2(p0, p1));
               if constexpr (FP8P) {
-                uint32_t nz;
-                const float2 sp = fmul2(make_float2(p0, p1), make_float2(a.p_scale, a.p_scale));
-                pk[e] = e4m3_cast_bf16x2(sp.x, sp.y, nz);
-                nzacc += nz;
-                if (count_each) {
-                  const int k0 = kbase + h * 2 * PC + 2 * e;
-                  const uint32_t f0 = (k0 <= lim && !(nz & 1u)) ? 1u : 0u;
-                  const uint32_t f1 = (k0 + 1 <= lim && !(nz >> 16)) ? 1u : 0u;
-                  fl_sink += (k0 < a.n_sink ? f0 : 0u) + (k0 + 1 < a.n_sink ? f1 : 0u);
-                  fl_non += (k0 < a.n_sink ? 0u : f0) + (k0 + 1 < a.n_sink ? 0u : f1);
-                }
+                uint32_t h2;
+                pk[e] = e4m3_round_bf16x2(p0, p1, h2);
+                if constexpr (COUNT) nz2 = count_nonzero_f16x2(h2, nz2);
               } else {
                 pk[e] = pack_bf16x2(p0, p1);
               }
             }
-            if constexpr (FP8P) {
-              if (a.stats != nullptr && plain_tile && row < N)
-                fl_non += 2u * PC - ((nzacc & 0xFFFFu) + (nzacc >> 16));
-            }
+            if constexpr (COUNT) nf_tile += f16x2_sum_u32(nz2);
             if constexpr (C::PV_SS) {
               // keys [2 PC h, 2 PC h + 2 PC) of row r in the 64-key boxes, 128-byte swizzle
               constexpr int CPB = 2 * PC / 8;  // 16-byte chunks per store group
@@ -511,6 +533,12 @@ __global__ void __launch_bounds__(320, 1)
               pk[e] = __float_as_uint(p);
             }
             tmem_st32(tS + h * 32, pk);
+          }
+        }
+        if constexpr (COUNT) {
+          if (row < N) {
+            nf_sink += nf_part;
+            nf_non += nf_tile - nf_part;
           }
         }
         // O correction after P is out (the S values are dead by now, which keeps
@@ -546,7 +574,8 @@ __global__ void __launch_bounds__(320, 1)
       if (ok) ok = mbar_wait(&bar_o[i], 0, &abort_sh, 12 + i);
       if (ok) {
         tc_fence_after();
-        const float inv = (C::EB == 1 ? a.sv[bh_kv] : 1.0f) / (l_run * a.p_scale);
+        // l_run is the sum of S p when P is cast (S = 1 otherwise)
+        const float inv = (C::EB == 1 ? a.sv[bh_kv] : 1.0f) / l_run;
         // output: fp32 for fp32 inputs, bf16 otherwise (also for E4M3 operands)
         using OutT = typename std::conditional<C::EB == 4, float, __nv_bfloat16>::type;
         OutT* orow = reinterpret_cast<OutT*>(a.o) + (static_cast<size_t>(bh) * N + row) * D;
@@ -576,25 +605,24 @@ __global__ void __launch_bounds__(320, 1)
             }
           }
         }
-        if (row < N) a.lse[static_cast<size_t>(bh) * N + row] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
+        if (row < N)
+          a.lse[static_cast<size_t>(bh) * N + row] = (m_run + log2f(l_run) - lg2S) * 0.69314718055994530942f;
       }
-      if constexpr (FP8P) {
-        if (a.stats != nullptr) {
-          // totals are exact counts of admissible keys for this row
-          uint32_t nk = 0;
-          if (row < N) nk = a.causal ? static_cast<uint32_t>(row + 1) : static_cast<uint32_t>(N);
-          const uint32_t ts = min(nk, static_cast<uint32_t>(max(a.n_sink, 0)));
-          const uint32_t tn = nk - ts;
-          const uint32_t v0 = __reduce_add_sync(0xffffffffu, fl_sink);
-          const uint32_t v1 = __reduce_add_sync(0xffffffffu, ts);
-          const uint32_t v2 = __reduce_add_sync(0xffffffffu, fl_non);
-          const uint32_t v3 = __reduce_add_sync(0xffffffffu, tn);
-          if (lane == 0) {
-            atomicAdd(a.stats + 0, static_cast<unsigned long long>(v0));
-            atomicAdd(a.stats + 1, static_cast<unsigned long long>(v1));
-            atomicAdd(a.stats + 2, static_cast<unsigned long long>(v2));
-            atomicAdd(a.stats + 3, static_cast<unsigned long long>(v3));
-          }
+      if constexpr (COUNT) {
+        // flushed = admissible keys of the row minus those whose P' stayed non-zero
+        uint32_t nk = 0;
+        if (row < N) nk = a.causal ? static_cast<uint32_t>(row + 1) : static_cast<uint32_t>(N);
+        const uint32_t ts = min(nk, static_cast<uint32_t>(max(a.n_sink, 0)));
+        const uint32_t tn = nk - ts;
+        const uint32_t v0 = __reduce_add_sync(0xffffffffu, ts - nf_sink);
+        const uint32_t v1 = __reduce_add_sync(0xffffffffu, ts);
+        const uint32_t v2 = __reduce_add_sync(0xffffffffu, tn - nf_non);
+        const uint32_t v3 = __reduce_add_sync(0xffffffffu, tn);
+        if (lane == 0) {
+          atomicAdd(a.stats + 0, static_cast<unsigned long long>(v0));
+          atomicAdd(a.stats + 1, static_cast<unsigned long long>(v1));
+          atomicAdd(a.stats + 2, static_cast<unsigned long long>(v2));
+          atomicAdd(a.stats + 3, static_cast<unsigned long long>(v3));
         }
       }
     }

@@ -11,6 +11,7 @@
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda.h>
 
 #ifndef FA_WAIT_LIMIT_NS
@@ -316,6 +317,43 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return d;
 }
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 A, B, D;\n\t"
+      "mov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\t"
+      "sub.rn.f32x2 D, A, B;\n\tmov.b64 {%0, %1}, D;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// 2^x of two values on the FMA and integer pipes, so that part of a softmax
+// tile's exponentials run beside the MUFU ex2 instead of queueing for it.
+// x is clamped to >= -126 (exponent field >= 1 after the shift below), split as
+// x = j + f with j = round-to-nearest(x) (adding 1.5 * 2^23 leaves j in the low
+// mantissa bits; subtracting it again gives j exactly, and x - j is exact) and
+// |f| <= 1/2; 2^f comes from a degree-3 polynomial and j is added to the
+// exponent field as an integer.  The polynomial is the minimax approximation of
+// 2^f on [-1/2, 1/2] in relative error, found with the Remez exchange algorithm
+// (equioscillation at five points); with these float32 coefficients its largest
+// relative error is 7.5e-5, below the 2^-9 half-ulp of the bf16 P it feeds.
+// Inputs are <= 127 (the softmax arguments here are <= 8).
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  constexpr float c0 = 0.99992805719375610f, c1 = 0.69326096773147583f, c2 = 0.24261112511157990f,
+                  c3 = 0.05517166852951050f;
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 kRound = make_float2(12582912.f, 12582912.f);  // 1.5 * 2^23
+  const float2 t = fadd2(x, kRound);
+  const float2 f = fsub2(x, fsub2(t, kRound));
+  float2 p = ffma2(make_float2(c3, c3), f, make_float2(c2, c2));
+  p = ffma2(p, f, make_float2(c1, c1));
+  p = ffma2(p, f, make_float2(c0, c0));
+  // t's bits are 0x4B400000 + j: shifted left by 23 only j remains, in the exponent field
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
 // three-input maximum (one instruction)
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
@@ -331,19 +369,32 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // E4M3 cast of two fp32 values (round to nearest even, saturating at +-448),
-// returned as bf16x2 bits without leaving the integer pipes for the widening:
-// E4M3 -> f16x2 is exact and every non-zero E4M3 value is an f16 normal, so the
-// bf16 bits are the f16 bits shifted right by 3 with the exponent rebiased
-// (+112 << 7); zero halves stay zero.  `nz` gets bit 0 / bit 16 set for
-// the halves that did not flush to zero.  Inputs must be >= 0.
-__device__ __forceinline__ uint32_t e4m3_cast_bf16x2(float lo, float hi, uint32_t& nz) {
+// returned as the bf16x2 pair of the same values, and `h2` = the same pair as
+// f16x2.  E4M3 -> f16x2 is exact and every non-zero E4M3 value (2^-9 .. 448) is
+// an f16 normal whose 7 lowest mantissa bits are zero, so h2 >> 3 holds each
+// value's sign, exponent field and top 7 mantissa bits in bf16 position; read as
+// bf16 that is the value times 2^(15-127), and one exact bf16x2 multiply by 2^112
+// restores it (zero stays zero).  Inputs must be >= 0.
+__device__ __forceinline__ uint32_t e4m3_round_bf16x2(float lo, float hi, uint32_t& h2) {
   uint16_t e;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(e) : "f"(hi), "f"(lo));
-  uint32_t h2;
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(e));
-  const uint32_t y = (h2 >> 3) & 0x0FFF0FFFu;
-  nz = ((y + 0x7FFF7FFFu) >> 15) & 0x00010001u;
-  return y + nz * 0x3800u;
+  uint32_t r;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(h2 >> 3), "r"(0x77807780u));
+  return r;
+}
+// Non-zero flags of an f16x2 pair of E4M3 values, added into an f16x2 counter:
+// a non-zero value is >= 2^-9, so 2^10 times it saturates to 1.0; zero stays 0.
+// Each half counts exactly up to 2048.
+__device__ __forceinline__ uint32_t count_nonzero_f16x2(uint32_t h2, uint32_t acc) {
+  uint32_t f, r;
+  asm("mul.rn.sat.f16x2 %0, %1, %2;" : "=r"(f) : "r"(h2), "r"(0x64006400u));
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(f), "r"(acc));
+  return r;
+}
+__device__ __forceinline__ uint32_t f16x2_sum_u32(uint32_t h2) {
+  const __half2 v = *reinterpret_cast<const __half2*>(&h2);
+  return static_cast<uint32_t>(__low2float(v) + __high2float(v));
 }
 
 // Wait used only on teardown paths: bounded by time, ignores the abort flag.

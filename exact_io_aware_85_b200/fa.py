@@ -28,6 +28,7 @@ lib.fa_status_string.restype = ctypes.c_char_p
 lib.fa_status_string.argtypes = [_ci]
 lib.fa_last_cuda_error.restype = _ci
 lib.fa_check_status.restype = _ci
+lib.fa_check_status.argtypes = [_vp]
 lib.fa_watchdog_selftest.argtypes = [ctypes.c_uint, _vp]
 
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_ALIGNMENT, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(6)
@@ -138,8 +139,10 @@ def fa_status_string(status: int) -> str:
     return lib.fa_status_string(int(status)).decode()
 
 
-def fa_check_status() -> int:
-    return int(lib.fa_check_status())
+def fa_check_status(stream=None) -> int:
+    """Status word of the current device once the work on `stream` (default:
+    torch's current stream) has finished; reading clears it."""
+    return int(lib.fa_check_status(_stream(stream)))
 
 
 def fa_last_cuda_error() -> int:

@@ -36,6 +36,7 @@ class Workload:
     sink: bool = False
     hkv: int = 0  # key/value heads for grouped-query attention (0: same as H)
     decode: bool = False  # one query row per head against an N-key cache
+    variant: str = ""  # sink workload: "" (P-cast with flush counts), "nostats", "bf16" (no cast)
 
     @property
     def scale(self) -> float:
@@ -72,6 +73,10 @@ WORKLOADS = {
     "train_d256": Workload("train_d256", 2, 8, 8192, 256, "bf16", True, backward=True),
     # the decoding step of "decode" at head dim 256
     "decode_d256": Workload("decode_d256", 8, 32, 32768, 256, "bf16", False, hkv=8, decode=True),
+    # the sink workload's P-cast without the flush counting, and the same inputs through the plain
+    # bf16 forward: together they split the P-cast's cost into the cast and the counting
+    "sink_nostats": Workload("sink_nostats", 1, 32, 16384, 128, "bf16", False, sink=True, variant="nostats"),
+    "sink_bf16": Workload("sink_bf16", 1, 32, 16384, 128, "bf16", False, sink=True, variant="bf16"),
 }
 
 SINK_DELTAS = (0.0, 2.0, 4.0, 6.0, 7.0, 8.0, 10.0, 12.0)

@@ -16,14 +16,18 @@
  *    LSE is the natural-log logsumexp of the scaled scores of each query row.
  *  - Sizes: B >= 1, H >= 1, N >= 1, d in {64, 128} (fa_fwd, fa_fwd_gqa, fa_bwd,
  *    fa_bwd_gqa, fa_bwd_noalloc and fa_decode also take d = 256, "FlashAttention
- *    (IT)", "FlashAttention-2 (2023)"); B*H*N*d < 2^31.
+ *    (IT)", "FlashAttention-2 (2023)").  Limits of the launches: N <= 2^30,
+ *    B*H < 2^31, B*H*ceil(N/128) < 2^31 and B*H*N*d < 2^40; element offsets
+ *    are 64-bit, so any size that fits in device memory within these is taken.
  *  - scale: the softmax scale (usually 1/sqrt(d)); finite and > 0.
  *  - causal != 0: query i attends to keys j <= i (square, top-left aligned);
  *    tiles that lie entirely in the future are skipped, never loaded.
- *  - Alignment: every device pointer 16-byte aligned.
+ *  - Alignment: every device pointer 16-byte aligned, except lse (4-byte:
+ *    the kernels write it one fp32 scalar at a time).
  *  - Ownership: the caller allocates and owns every buffer.  The library never
- *    allocates, frees or synchronises (fa_check_status excepted); all work is
- *    enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream).
+ *    allocates, frees or synchronises (fa_check_status synchronises the stream
+ *    it is given); all work is enqueued on `stream` (a cudaStream_t; NULL = the
+ *    legacy default stream).
  *  - Errors: invalid arguments are rejected before anything is launched and
  *    return a non-zero fa_status; there is no fallback path.  A failed launch
  *    returns FA_ERR_CUDA (fa_last_cuda_error() gives the cudaError_t).  Device
@@ -49,8 +53,13 @@ extern "C" {
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, bad scale/S/kv_order */
-  FA_ERR_UNSUPPORTED = 2, /* head dim other than 64/128, or sizes over the limits */
-  FA_ERR_ALIGNMENT = 3,   /* a pointer that is not 16-byte aligned */
+  FA_ERR_UNSUPPORTED = 2, /* a head dim the entry point does not take (64 and 128
+                             everywhere; 256 only where its comment says so), sizes
+                             over the limits above, B*H_kv > 65535 (fa_decode) or
+                             B*H > 65535 (fa_fp8_quantize), more than 16 query heads
+                             per key/value head (fa_decode), or a workspace larger
+                             than FA_BWD_NOALLOC_MAX_BYTES (fa_bwd_noalloc) */
+  FA_ERR_ALIGNMENT = 3,   /* a pointer without the alignment the conventions require */
   FA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed */
   FA_ERR_TIMEOUT = 5      /* a device-side wait gave up (reported by fa_check_status) */
 } fa_status;
@@ -60,9 +69,11 @@ typedef enum {
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d, int causal,
            float scale, void* stream);
 
-/* Forward, fp32 in/out: the same algorithm on the tf32 tensor-core path
- * (operands rounded to tf32 by the tensor core, fp32 accumulation, fp32 softmax).
- * q, k, v, o: fp32 [B,H,N,d]; lse: fp32 [B,H,N]. */
+/* Forward, fp32 in/out: the same algorithm on the tf32 tensor-core path.  Q and
+ * K are rounded to tf32 (round to nearest even) in shared memory before S = Q K^T,
+ * so the scores carry no truncation bias; V and P enter P V as the tensor core
+ * reads them (their low 13 mantissa bits are ignored).  fp32 accumulation and
+ * fp32 softmax.  d = 64 only.  q, k, v, o: fp32 [B,H,N,d]; lse: fp32 [B,H,N]. */
 int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int H, int N, int d,
                int causal, float scale, void* stream);
 
@@ -91,8 +102,10 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
  *  - Sizes whose workspace (fa_bwd_workspace_bytes) exceeds that maximum are
  *    rejected with FA_ERR_UNSUPPORTED before anything is launched.
  *  - The first call on a device looks up that device's address of the array
- *    (cudaGetSymbolAddress) and caches it; make that first call before any
- *    stream capture.
+ *    (cudaGetSymbolAddress, with the device current) and caches it with the id
+ *    of the CUDA context; a call in another context (after a device reset, for
+ *    one) looks it up again.  Make the first call on a device before any stream
+ *    capture.
  *  - All calls on a device share the one array and it keeps the previous call's
  *    contents; each call rewrites every part it reads (the first of its kernels
  *    rewrites the row statistics and zeroes the dQ accumulator).  Calls whose
@@ -179,10 +192,14 @@ const char* fa_status_string(int status);
 /* The cudaError_t of the last FA_ERR_CUDA returned on this host thread. */
 int fa_last_cuda_error(void);
 
-/* Synchronises the current device, then reads and clears the device status word:
- * FA_OK, or FA_ERR_TIMEOUT if a kernel's bounded wait gave up since the last
- * call (FA_ERR_CUDA if the synchronisation itself failed). */
-int fa_check_status(void);
+/* Reads the device status word after the work on `stream` has finished (a copy
+ * enqueued on `stream`, then cudaStreamSynchronize(stream); NULL = the legacy
+ * default stream, which also waits for the other blocking streams), and clears
+ * it: FA_OK, or FA_ERR_TIMEOUT if a bounded wait in a kernel of this library gave
+ * up on the current device since the last call (FA_ERR_CUDA if a copy or the
+ * synchronisation failed).  The word is per device, not per stream: a timeout
+ * raised by work on another stream is reported too, once that work is done. */
+int fa_check_status(void* stream);
 
 /* Failure-path self-test: launches a one-block kernel whose bounded wait on a
  * barrier that nothing signals gives up after limit_us microseconds (1 .. 10^7),

@@ -118,3 +118,37 @@ def test_head_dim_256_is_admitted_where_declared(lib):
     assert lib.fa_decode(good, good, good, good, good, 1, 32, 1, 64, 256, 0.1, good, 1 << 30, None) == 2  # g > 16
     lib.fa_fwd_fp8.argtypes = [vp] * 3 + [vp] * 3 + [vp, vp] + [ci] * 5 + [cf, cf, ci, vp]
     assert lib.fa_fwd_fp8(*([good] * 8), 1, 1, 64, 256, 1, 0.1, 256.0, 0, None) == 2      # FP8 takes d = 128
+
+
+def test_size_limits_and_lse_alignment(lib):
+    """Sizes are limited by what the launches express, not by a 2^31-element
+    cap; lse needs 4-byte alignment only.  Every call here stops at a later
+    argument check (an invalid S), so nothing is launched on the fake pointers:
+    status 1 shows the earlier checks passed."""
+    vp, ci, cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.fa_fwd_fp8p.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, cf, ci, vp, ci, vp]
+    good = vp(1 << 20)
+
+    def call(B, H, N, d=128, lse=good):
+        return lib.fa_fwd_fp8p(good, good, good, good, lse, B, H, N, d, 0, 0.1, -1.0, 0, None, 4, None)
+
+    assert call(4, 32, 131072) == 1             # 2^31 elements: a long-context prefill is taken
+    assert call(1, 1, (1 << 30) + 1, 64) == 2   # N past 2^30
+    assert call(65536, 32768, 1) == 2           # B*H = 2^31
+    assert call(1 << 14, 1 << 14, 128, 64) == 2  # 2^28 CTAs would fit, but 2^41 elements do not
+    assert call(1 << 10, 1 << 10, 128, 64) == 1  # 2^20 heads, 2^33 elements: taken
+    assert call(1, 1, 64, lse=vp((1 << 20) + 4)) == 1   # lse 4-byte aligned: accepted
+    assert call(1, 1, 64, lse=vp((1 << 20) + 2)) == 3   # lse 2-byte aligned: refused
+
+
+def test_grid_y_limits_refused_before_launch(lib):
+    """fa_decode puts B*H_kv and fa_fp8_quantize puts B*H on gridDim.y (at most
+    65535); larger counts are refused before any launch."""
+    vp, ci, cf, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    good = vp(1 << 20)
+    lib.fa_decode.argtypes = [vp] * 5 + [ci] * 5 + [cf, vp, sz, vp]
+    assert lib.fa_decode(good, good, good, good, good, 1024, 128, 128, 1, 64, 0.1, good, 1 << 40, None) == 2
+    assert lib.fa_decode(good, good, good, good, good, 1023, 128, 64, 1, 64, 0.1, good, 10, None) == 1  # 65472: short workspace next
+    lib.fa_fp8_quantize.argtypes = [vp] * 4 + [vp] * 3 + [vp] * 3 + [ci] * 4 + [vp]
+    assert lib.fa_fp8_quantize(*([good] * 10), 256, 256, 1, 64, None) == 2
+    assert lib.fa_fp8_quantize(*([good] * 10), 1, 1, 64, 96, None) == 2

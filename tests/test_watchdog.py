@@ -24,3 +24,13 @@ def test_unsignalled_wait_times_out_and_context_survives():
     torch.cuda.synchronize()
     assert fa.fa_check_status() == fa.FA_OK
     assert torch.isfinite(o.float()).all()
+
+
+def test_status_is_read_after_the_given_stream():
+    """fa_check_status(stream) waits for that stream only; a timeout raised by a
+    kernel on a side stream is reported once that stream's work is done."""
+    from exact_io_aware_85_b200 import fa
+    side = torch.cuda.Stream()
+    fa.fa_watchdog_selftest(20000, stream=side)
+    assert fa.fa_check_status(side) == fa.FA_ERR_TIMEOUT
+    assert fa.fa_check_status(side) == fa.FA_OK
