@@ -356,9 +356,12 @@ def main():
     small = 3 * q.numel() * q.element_size() < 126e6
     flush = torch.empty(int(256e6), dtype=torch.uint8, device="cuda") if small else None
 
+    nvtx = torch.cuda.nvtx  # ranges for an external profiler's timeline: warm-up, timed steps, end-to-end steps
+    nvtx.range_push(f"fa_bench:{w.name}:warmup")
     for _ in range(max(3, args.warmup)):
         run()
     torch.cuda.synchronize()
+    nvtx.range_pop()
     assert fa.fa_check_status() == 0
 
     # ---- device-resident timing: per-launch CUDA events on the launch stream ----
@@ -369,6 +372,7 @@ def main():
     with ClockSampler(local) as clk:
         t_all0 = torch.cuda.Event(enable_timing=True)
         t_all1 = torch.cuda.Event(enable_timing=True)
+        nvtx.range_push(f"fa_bench:{w.name}:timed x{args.steps}")
         t_all0.record(stream)
         for i in range(args.steps):
             if flush is not None:
@@ -378,6 +382,7 @@ def main():
             ends[i].record(stream)
         t_all1.record(stream)
         torch.cuda.synchronize()
+        nvtx.range_pop()
     barrier(ws)
     launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     step_ms_local = sum(launch_ms) / len(launch_ms)
@@ -418,11 +423,13 @@ def main():
     barrier(ws)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    nvtx.range_push(f"fa_bench:{w.name}:e2e x{e2e_steps}")
     e0.record(stream)
     for _ in range(e2e_steps):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
+    nvtx.range_pop()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, ws)
     h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
     d2h = (3 * q.numel() * q.element_size() if w.backward else o.numel() * o.element_size()) + lse.numel() * 4

@@ -126,6 +126,10 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   if ((st = encode_qkv_map(&mv, v, dt, sizeof(T), D, N, B * Hkv,
                            sizeof(T) == 4 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
     return st;
+  // O leaves by TMA store when the operands are bf16 (the map is unused otherwise)
+  CUtensorMap mo = mq;
+  if (sizeof(T) == 2 && (st = encode_qkv_map(&mo, o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, N, BH)) != FA_OK)
+    return st;
   fa::FwdArgs a;
   a.o = o;
   a.lse = lse;
@@ -146,8 +150,15 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   auto kern = fa::fa_fwd_kernel<T, D, FP8P, COUNT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_fail(e);
+  // the softmax warpgroups raise their budget out of the block's launch
+  // allocation (setmaxnreg); with fewer registers at launch the raise would
+  // wait forever, so such a build is refused here
+  cudaFuncAttributes fattr;
+  e = cudaFuncGetAttributes(&fattr, kern);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (fattr.numRegs < C::LAUNCH_REGS) return FA_ERR_UNSUPPORTED;
   const long long grid = static_cast<long long>(a.nblk) * BH;
-  kern<<<static_cast<unsigned>(grid), C::NTHREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, a);
+  kern<<<static_cast<unsigned>(grid), C::NTHREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return FA_OK;
@@ -196,7 +207,21 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.causal = causal ? 1 : 0;
-  if constexpr (D != 64) {
+  if constexpr (D == 128) {
+    // 128-query steps (Q and dO tiles of 128 rows)
+    using CQ = fa::BwdQ128Cfg;
+    auto kern = fa::fa_bwd_main_q128_kernel;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, CQ::SMEM_BYTES);
+    if (e != cudaSuccess) return cuda_fail(e);
+    // the gradient warpgroups raise their budget out of the launch allocation
+    // (setmaxnreg): refuse a build whose launch register count is too small
+    cudaFuncAttributes fattr;
+    e = cudaFuncGetAttributes(&fattr, kern);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (fattr.numRegs < CQ::LAUNCH_REGS) return FA_ERR_UNSUPPORTED;
+    kern<<<static_cast<unsigned>(static_cast<long long>(n_tiles) * BHkv), CQ::NTHREADS, CQ::SMEM_BYTES, stream>>>(
+        mq, mk, mv, mdo, a);
+  } else if constexpr (D != 64) {
     // 64-query variant: Q and dO tiles of 64 rows; at d = 256 two CTAs per key
     // tile, one per 128-column slice of dV, dK and dQ
     CUtensorMap mq64, mdo64;
@@ -220,8 +245,10 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   if (e != cudaSuccess) return cuda_fail(e);
   // 3. dQ accumulator -> bf16
   const long long vecs = static_cast<long long>(BH) * N * (D / 8);
+  // the 128-query pass at d = 128 accumulates dS / scale (its dK epilogue and this
+  // pass apply the scale); the others accumulate dS
   fa::fa_bwd_post_kernel<D><<<static_cast<unsigned>((vecs + 255) / 256), 256, 0, stream>>>(
-      dq_acc, static_cast<__nv_bfloat16*>(dq), N, npad, vecs);
+      dq_acc, static_cast<__nv_bfloat16*>(dq), N, npad, vecs, D == 128 ? scale : 1.0f);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return FA_OK;

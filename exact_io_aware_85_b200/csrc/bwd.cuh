@@ -74,12 +74,13 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __
 }
 
 // ---------------------------------------------------------------------------
-// bwd_post: dQ accumulator (fp32, padded rows) -> bf16
+// bwd_post: dQ accumulator (fp32, padded rows) times f -> bf16 (f is the
+// softmax scale when the main pass accumulated dS / scale, 1 otherwise)
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_post_kernel(const float* __restrict__ dq_acc,
                                                           __nv_bfloat16* __restrict__ dq, int N, int Npad,
-                                                          long long vec_total) {
+                                                          long long vec_total, float f) {
   const long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;  // one 8-element vector
   if (g >= vec_total) return;
   constexpr int VPR = D / 8;
@@ -90,10 +91,10 @@ __global__ void __launch_bounds__(256) fa_bwd_post_kernel(const float* __restric
   const float4* src = reinterpret_cast<const float4*>(dq_acc + (static_cast<size_t>(bh) * Npad + n) * D + part * 8);
   const float4 a = src[0], b = src[1];
   uint4 w;
-  w.x = pack_bf16x2(a.x, a.y);
-  w.y = pack_bf16x2(a.z, a.w);
-  w.z = pack_bf16x2(b.x, b.y);
-  w.w = pack_bf16x2(b.z, b.w);
+  w.x = pack_bf16x2(a.x * f, a.y * f);
+  w.y = pack_bf16x2(a.z * f, a.w * f);
+  w.z = pack_bf16x2(b.x * f, b.y * f);
+  w.w = pack_bf16x2(b.z * f, b.w * f);
   *reinterpret_cast<uint4*>(dq + static_cast<size_t>(row) * D + part * 8) = w;
 }
 
@@ -135,6 +136,12 @@ struct BwdCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
+// dst[0..3] += v[0..3] (fp32) as one 16-byte reduction in the L2
+__device__ __forceinline__ void red_add_v4(float* dst, const uint32_t* v) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(__uint_as_float(v[0])),
+               "f"(__uint_as_float(v[1])), "f"(__uint_as_float(v[2])), "f"(__uint_as_float(v[3]))
+               : "memory");
+}
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -883,6 +890,406 @@ __global__ void __launch_bounds__(448, 1)
   if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// bwd_main at d = 128 with 128-query steps
+// ---------------------------------------------------------------------------
+// One CTA per (128-key tile, key/value head), K_j and V_j resident.  Each step
+// takes 128 queries, so S^T, dP^T and dQ^T are N = 128 MMAs (a shared-memory
+// MMA costs about the same ~110 cycles per 16-deep step at N = 64 as at N = 128,
+// so this halves their cost per FLOP against 64-query steps).  Tensor memory
+// holds one step (dV, dK, S^T, dP^T: all 512 columns), so the step's hand-offs
+// are split finely enough that the tensor core stays busy:
+//   S^T(t) -> [gradient warps: P]  dP^T(t) -> [gradient warps: dS]
+//   dV(t) as soon as P^T is stored (while dS is computed), dK(t) once dS^T is
+//   stored, dQ^T(t) into the dP^T columns (after dK has read dS^T there), then
+//   S^T(t+1) while the drain warps empty dQ^T(t), then dP^T(t+1).
+// The gradient warps read neither LSE nor D: the accumulators start from them.
+// Before S^T(t) the drain warps fill the S^T columns with -LSE_q / scale (one
+// row per key, every row the same) and before dP^T(t) the dP^T columns with
+// -D_q, and the two MMAs accumulate onto them, so the gradient warps compute
+// P = 2^(scale log2(e) acc) and dS = P acc' straight from tensor memory.  The
+// softmax scale of dS is applied to dK in its epilogue and to dQ in the post
+// pass.  dQ^T(t) is drained with coalesced fp32 reductions (a warp adds 32
+// consecutive head-dimension entries of one query row).
+// Warp roles (16 warps; registers per thread after setmaxnreg):
+//   warps 0-7   gradient warps (144): thread = key row (TMEM lane); warps 0-3
+//               queries 0-63 of the step, warps 4-7 queries 64-127
+//   warps 8-11  dQ drain and accumulator set-up (152): thread = TMEM lane
+//   warp  12    TMA producer, warp 13 MMA issuer and TMEM owner, 14-15 idle (72)
+// Launched at 128 registers a thread: 2 x 128 x 144 + 128 x 152 + 128 x 72 =
+// 65536 = 512 x 128, and 144 + 144 + 152 + 72 = 512 per sub-partition.
+struct BwdQ128Cfg {
+  static constexpr int D = 128;
+  static constexpr int BOX = 16384;             // 128 rows x 128 bytes
+  static constexpr int TILE = 2 * BOX;          // 128 rows x 128 bf16 columns
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + TILE;
+  static constexpr int NST = 2;                 // Q/dO/LSE/D load stages
+  static constexpr int OFF_Q = OFF_V + TILE;
+  static constexpr int OFF_DO = OFF_Q + NST * TILE;
+  static constexpr int OFF_DS = OFF_DO + NST * TILE;  // dS^T: 128 keys x 128 queries, two 64-query blocks
+  static constexpr int OFF_LSE = OFF_DS + TILE;       // NST x 128 floats
+  static constexpr int OFF_DV = OFF_LSE + NST * 512;  // NST x 128 floats
+  static constexpr int OFF_BAR = OFF_DV + NST * 512;
+  static constexpr int SMEM_BYTES = OFF_BAR + 256;
+  static constexpr uint32_t COL_DV = 0, COL_DK = 128, COL_S = 256, COL_DP = 384;
+  static constexpr int NTHREADS = 512;
+  static constexpr int LAUNCH_REGS = 128, GRAD_REGS = 144, DRAIN_REGS = 152, OTHER_REGS = 72;
+  static_assert(2 * 128 * GRAD_REGS + 128 * DRAIN_REGS + 128 * OTHER_REGS <= NTHREADS * LAUNCH_REGS,
+                "register split");
+  static_assert(2 * GRAD_REGS + DRAIN_REGS + OTHER_REGS <= 512, "registers per sub-partition");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+__global__ void __launch_bounds__(512, 1)
+    fa_bwd_main_q128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                            const BwdArgs a) {
+  using C = BwdQ128Cfg;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* bar_kv = bars + 0;
+  uint64_t* bar_ld_full = bars + 1;   // [NST]
+  uint64_t* bar_ld_empty = bars + 3;  // [NST]
+  uint64_t* bar_s_full = bars + 5;
+  uint64_t* bar_dp_full = bars + 6;
+  uint64_t* bar_p_ready = bars + 7;   // 256 arrivals: P^T stored, S^T read
+  uint64_t* bar_ds_ready = bars + 8;  // 256 arrivals: dS^T stored (tensor and shared memory)
+  uint64_t* bar_dq_full = bars + 9;   // dQ^T(t) complete (also: shared dS^T read)
+  uint64_t* bar_dp_init = bars + 10;  // 128 arrivals: dQ^T(t-1) read out, -D(t) in the dP^T columns
+  uint64_t* bar_s_free = bars + 15;   // dV(t) complete: the S^T columns may be refilled
+  uint64_t* bar_s_init = bars + 16;   // 128 arrivals: -LSE(t) / scale in the S^T columns
+  uint64_t* bar_acc = bars + 11;
+  uint64_t* bar_done = bars + 12;
+  uint32_t* tmem_base_sh = reinterpret_cast<uint32_t*>(bars + 13);
+  volatile int* abort_sh = reinterpret_cast<volatile int*>(bars + 14);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int N = a.N;
+  const int bh_kv = blockIdx.x % a.BHkv;  // key/value head
+  const int j = blockIdx.x / a.BHkv;      // key tile; j = 0 (the longest walk when causal) first
+  const int i0 = a.causal ? j : 0;        // first query tile of 128
+  const int spq = a.n_tiles - i0;         // query tiles per query head
+  const int steps = spq * a.group;        // the walk covers every query head of the group
+  auto step_head = [&](int t) { return bh_kv * a.group + t / spq; };
+  auto step_tile = [&](int t) { return i0 + t % spq; };
+
+  // the swizzled TMA/UMMA layouts need a 1024-byte aligned base (uniform: every
+  // thread returns before any barrier)
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicCAS(&g_fa_status, 0, 4 /*FA_ERR_CUDA*/ | (97 << 8));
+    return;
+  }
+  if (warp == 13) {
+    tmem_alloc(tmem_base_sh, 512);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    *abort_sh = 0;
+    mbar_init(bar_kv, 1);
+    for (int b = 0; b < C::NST; ++b) {
+      mbar_init(bar_ld_full + b, 1);
+      mbar_init(bar_ld_empty + b, 1);
+    }
+    mbar_init(bar_s_full, 1);
+    mbar_init(bar_dp_full, 1);
+    mbar_init(bar_p_ready, 256);
+    mbar_init(bar_ds_ready, 256);
+    mbar_init(bar_dq_full, 1);
+    mbar_init(bar_dp_init, 128);
+    mbar_init(bar_s_free, 1);
+    mbar_init(bar_s_init, 128);
+    mbar_init(bar_acc, 1);
+    mbar_init(bar_done, 1);
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_base_sh;
+
+  if (warp >= 12) {
+    setmaxnreg_to<C::LAUNCH_REGS, C::OTHER_REGS>();
+    if (warp == 12 && lane == 0) {
+      // ============================ producer ===================================
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmDO);
+      mbar_arrive_expect_tx(bar_kv, 2 * C::TILE);
+      for (int b = 0; b < 2; ++b) {
+        tma_load_3d(smem + C::OFF_K + b * C::BOX, &tmK, bar_kv, b * 64, j * 128, bh_kv);
+        tma_load_3d(smem + C::OFF_V + b * C::BOX, &tmV, bar_kv, b * 64, j * 128, bh_kv);
+      }
+      int t = 0;
+      for (; t < steps; ++t) {
+        const int i = step_tile(t), hq = step_head(t);
+        const int s = t % C::NST;
+        const uint32_t ph = (t / C::NST) & 1;
+        if (!mbar_wait_inl(bar_ld_empty + s, ph ^ 1, abort_sh, 80)) break;
+        mbar_arrive_expect_tx(bar_ld_full + s, 2 * C::TILE + 1024);
+        for (int b = 0; b < 2; ++b) {
+          tma_load_3d(smem + C::OFF_Q + s * C::TILE + b * C::BOX, &tmQ, bar_ld_full + s, b * 64, i * 128, hq);
+          tma_load_3d(smem + C::OFF_DO + s * C::TILE + b * C::BOX, &tmDO, bar_ld_full + s, b * 64, i * 128, hq);
+        }
+        const size_t roff = static_cast<size_t>(hq) * a.Npad + static_cast<size_t>(i) * 128;
+        bulk_load(smem + C::OFF_LSE + s * 512, a.lse2 + roff, 512, bar_ld_full + s);
+        bulk_load(smem + C::OFF_DV + s * 512, a.dvec + roff, 512, bar_ld_full + s);
+      }
+      mbar_wait_drain(bar_kv, 0, 100000000ull);
+      for (int u = max(0, t - C::NST); u < t; ++u)
+        mbar_wait_drain(bar_ld_full + u % C::NST, (u / C::NST) & 1, 100000000ull);
+    } else if (warp == 13 && lane == 0) {
+      // ============================ MMA issuer =================================
+      constexpr uint32_t id_s = make_idesc(128, 128, kFmtBF16, 0, 0);  // S^T, dP^T: N = 128 queries
+      constexpr uint32_t id_g = make_idesc(128, 128, kFmtBF16, 0, 1);  // dV, dK: B MN-major (d contiguous)
+      constexpr uint32_t id_q = make_idesc(128, 128, kFmtBF16, 1, 1);  // dQ^T: A = K^T, B = dS^T, MN-major
+      const uint32_t k_addr = smem_u32(smem + C::OFF_K), v_addr = smem_u32(smem + C::OFF_V);
+      const uint32_t q_addr = smem_u32(smem + C::OFF_Q), do_addr = smem_u32(smem + C::OFF_DO);
+      const uint32_t ds_addr = smem_u32(smem + C::OFF_DS);
+      bool ok = mbar_wait_inl(bar_kv, 0, abort_sh, 81);
+      for (int t = 0; ok && t < steps; ++t) {
+        const int st = t % C::NST;
+        const uint32_t ph = t & 1;
+        if (!(ok = mbar_wait_inl(bar_ld_full + st, (t / C::NST) & 1, abort_sh, 82))) break;
+        tc_fence_after();
+        const uint32_t qa = q_addr + st * C::TILE, da = do_addr + st * C::TILE;
+        // S^T = -LSE/scale + K_j Q_i^T (M = 128 keys, N = 128 queries, K = d), onto
+        // the drain warps' fill of the columns that dV(t-1) read last
+        if (!(ok = mbar_wait_inl(bar_s_init, ph, abort_sh, 91))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t off = (k >> 2) * C::BOX + (k & 3) * 32;
+          mma_ss(tmem + C::COL_S, make_sdesc_sw128(k_addr + off, 16, 1024), make_sdesc_sw128(qa + off, 16, 1024),
+                 id_s, 1u);
+        }
+        mma_commit(bar_s_full);
+        // dP^T = -D + V_j dO_i^T, onto the fill that replaced dQ^T(t-1)
+        if (!(ok = mbar_wait_inl(bar_dp_init, ph, abort_sh, 83))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t off = (k >> 2) * C::BOX + (k & 3) * 32;
+          mma_ss(tmem + C::COL_DP, make_sdesc_sw128(v_addr + off, 16, 1024), make_sdesc_sw128(da + off, 16, 1024),
+                 id_s, 1u);
+        }
+        mma_commit(bar_dp_full);
+        // dV += P^T dO_i (M = 128 keys, N = 128 columns, K = 128 queries): P^T in
+        // tensor memory, each 64-query half packed in the first 32 of its 64 columns
+        if (!(ok = mbar_wait_inl(bar_p_ready, ph, abort_sh, 84))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          mma_ts(tmem + C::COL_DV, tmem + C::COL_S + 64 * (k >> 2) + 8 * (k & 3),
+                 make_sdesc_sw128(da + k * 2048, C::BOX, 1024), id_g, (t > 0 || k > 0) ? 1u : 0u);
+        mma_commit(bar_s_free);  // P^T read: the S^T columns may be refilled
+        // dK += dS^T Q_i (dS^T likewise over dP^T)
+        if (!(ok = mbar_wait_inl(bar_ds_ready, ph, abort_sh, 85))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + 64 * (k >> 2) + 8 * (k & 3),
+                 make_sdesc_sw128(qa + k * 2048, C::BOX, 1024), id_g, (t > 0 || k > 0) ? 1u : 0u);
+        mma_commit(bar_ld_empty + st);  // Q_i, dO_i, LSE_i, D_i read by everything that needs them
+        // dQ_i^T = K_j^T dS^T (M = 128 columns, N = 128 queries, K = 128 keys) into
+        // the dP^T columns, after dK has read dS^T there
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          mma_ss(tmem + C::COL_DP, make_sdesc_sw128(k_addr + k * 2048, C::BOX, 1024),
+                 make_sdesc_sw128(ds_addr + k * 2048, C::BOX, 1024), id_q, k > 0 ? 1u : 0u);
+        mma_commit(bar_dq_full);
+      }
+      if (ok) mma_commit(bar_acc);
+      mma_commit(bar_done);
+      mbar_wait_drain(bar_done, 0, 100000000ull);
+    }
+    tc_fence_before();
+    named_bar_sync_all(1, C::NTHREADS);
+    if (warp == 13) {
+      __syncwarp();  // lane 0 issued the MMAs alone: reconverge for the warp-wide dealloc
+      tc_fence_after();
+      tmem_dealloc(tmem, 512);
+    }
+  } else if (warp >= 8) {
+    setmaxnreg_to<C::LAUNCH_REGS, C::DRAIN_REGS>();
+    // ============================ dQ drain and accumulator set-up ===========
+    // Per step t: fill the S^T columns with -LSE(t)/scale once dV(t-1) has read
+    // P^T there; read dQ^T(t-1) out of the dP^T columns (thread = head-dimension
+    // column c, one value per query), fill them with -D(t), release them, and
+    // only then add dQ^T(t-1) into the accumulator (the reductions queue behind
+    // nothing that the next MMAs wait for).
+    const int c = threadIdx.x - 256;  // TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    const float neg_inv_c = -1.0f / a.scale_log2;  // -LSE log2(e) / (scale log2(e)) = -LSE / scale
+    bool ok = true;
+    for (int t = 0; t <= steps && ok; ++t) {
+      const bool fill = t < steps;
+      const int st = t % C::NST;
+      if (fill) {
+        // -LSE(t)/scale into the S^T columns once dV(t-1) has read P^T(t-1)
+        if (!(ok = mbar_wait_inl(bar_ld_full + st, (t / C::NST) & 1, abort_sh, 92))) break;
+        if (t >= 1 && !(ok = mbar_wait_inl(bar_s_free, (t - 1) & 1, abort_sh, 93))) break;
+        tc_fence_after();
+        const float4* l4p = reinterpret_cast<const float4*>(smem + C::OFF_LSE + st * 512);
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {  // 16 columns (queries) per store
+          uint32_t w[16];
+#pragma unroll
+          for (int e4 = 0; e4 < 4; ++e4) {
+            const float4 l4 = l4p[4 * ch + e4];
+            w[4 * e4 + 0] = __float_as_uint(l4.x * neg_inv_c);
+            w[4 * e4 + 1] = __float_as_uint(l4.y * neg_inv_c);
+            w[4 * e4 + 2] = __float_as_uint(l4.z * neg_inv_c);
+            w[4 * e4 + 3] = __float_as_uint(l4.w * neg_inv_c);
+          }
+          tmem_st16(tmem + lane_base + C::COL_S + 16 * ch, w);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar_s_init);
+      }
+      uint32_t v[128];
+      if (t >= 1) {
+        if (!(ok = mbar_wait_inl(bar_dq_full, (t - 1) & 1, abort_sh, 86))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch)
+          tmem_ld32(tmem + lane_base + C::COL_DP + 32 * ch, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * ch]));
+        tmem_wait_ld();
+      }
+      if (fill) {
+        const float4* d4p = reinterpret_cast<const float4*>(smem + C::OFF_DV + st * 512);
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          uint32_t w[16];
+#pragma unroll
+          for (int e4 = 0; e4 < 4; ++e4) {
+            const float4 d4 = d4p[4 * ch + e4];
+            w[4 * e4 + 0] = __float_as_uint(-d4.x);
+            w[4 * e4 + 1] = __float_as_uint(-d4.y);
+            w[4 * e4 + 2] = __float_as_uint(-d4.z);
+            w[4 * e4 + 3] = __float_as_uint(-d4.w);
+          }
+          tmem_st16(tmem + lane_base + C::COL_DP + 16 * ch, w);
+        }
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      if (fill) mbar_arrive(bar_dp_init);
+      if (t >= 1) {
+        const int i = step_tile(t - 1), hq = step_head(t - 1);
+        float* dst = a.dq_acc + (static_cast<size_t>(hq) * a.Npad + static_cast<size_t>(i) * 128) * C::D + c;
+#pragma unroll
+        for (int q = 0; q < 128; ++q) atomicAdd(dst + static_cast<size_t>(q) * C::D, __uint_as_float(v[q]));
+      }
+    }
+    tc_fence_before();
+    named_bar_sync_all(1, C::NTHREADS);
+  } else {
+    setmaxnreg_to<C::LAUNCH_REGS, C::GRAD_REGS>();
+    // ============================ gradient warps =============================
+    const int half = warp >> 2;       // queries [64 half, 64 half + 64) of each step
+    const int r = threadIdx.x & 127;  // key row in tile == TMEM lane
+    const int key = j * 128 + r;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    const float cl = a.scale_log2;
+    bool ok = true;
+    for (int t = 0; t < steps && ok; ++t) {
+      const int i = step_tile(t);
+      const uint32_t ph = t & 1;
+      const int q0 = i * 128 + half * 64;
+      const bool need_mask = (a.causal && q0 < j * 128 + 128) || key >= N;
+      // ---- P = exp2(scale log2(e) (S^T - LSE / scale)) for 64 queries; P^T to TMEM
+      if (!(ok = mbar_wait_inl(bar_s_full, ph, abort_sh, 87))) break;
+      tc_fence_after();
+      float p[64];
+#pragma unroll
+      for (int sub = 0; sub < 2; ++sub) {
+        float* ps = p + 32 * sub;
+        tmem_ld32(tmem + lane_base + C::COL_S + 64 * half + 32 * sub, *reinterpret_cast<uint32_t(*)[32]>(ps));
+        tmem_wait_ld();
+#pragma unroll
+        for (int e2 = 0; e2 < 16; ++e2) {
+          const float2 x = fmul2(make_float2(ps[2 * e2], ps[2 * e2 + 1]), make_float2(cl, cl));
+          ps[2 * e2] = ex2_approx(x.x);
+          ps[2 * e2 + 1] = ex2_approx(x.y);
+        }
+        if (need_mask) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (key >= N || (a.causal && key > q0 + 32 * sub + e)) ps[e] = 0.f;
+        }
+        // P^T (bf16, two per column) into columns 16 sub .. 16 sub + 15 of this
+        // half: their fp32 scores have been read already
+        uint32_t pw[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) pw[e] = pack_bf16x2(ps[2 * e], ps[2 * e + 1]);
+        tmem_st16(tmem + lane_base + C::COL_S + 64 * half + 16 * sub, pw);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_p_ready);
+      // ---- dS / scale = P (dP - D); dS^T to TMEM (A of dK) and shared memory (B of dQ^T)
+      if (!(ok = mbar_wait_inl(bar_dp_full, ph, abort_sh, 88))) break;
+      tc_fence_after();
+      // the shared dS^T buffer was last read by dQ(t-1)
+      if (t >= 1 && !(ok = mbar_wait_inl(bar_dq_full, ph ^ 1, abort_sh, 89))) break;
+      uint8_t* db = smem + C::OFF_DS + half * C::BOX;  // this half's 64-query block
+#pragma unroll
+      for (int sub = 0; sub < 2; ++sub) {
+        uint32_t dp[32];
+        tmem_ld32(tmem + lane_base + C::COL_DP + 64 * half + 32 * sub, dp);
+        tmem_wait_ld();
+        uint32_t dw[16];
+#pragma unroll
+        for (int e2 = 0; e2 < 16; ++e2) {  // the dP^T accumulator started from -D
+          const float* ps = p + 32 * sub + 2 * e2;
+          const float2 g = fmul2(make_float2(ps[0], ps[1]),
+                                 make_float2(__uint_as_float(dp[2 * e2]), __uint_as_float(dp[2 * e2 + 1])));
+          dw[e2] = pack_bf16x2(g.x, g.y);
+        }
+        tmem_st16(tmem + lane_base + C::COL_DP + 64 * half + 16 * sub, dw);
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {  // 16-byte chunk 4 sub + cc (8 queries) of row r
+          const uint32_t off = sw128_off(r, 4 * sub + cc);
+          *reinterpret_cast<uint4*>(db + off) = make_uint4(dw[4 * cc], dw[4 * cc + 1], dw[4 * cc + 2], dw[4 * cc + 3]);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      fence_proxy_async_smem();
+      mbar_arrive(bar_ds_ready);
+    }
+    // ---- epilogue: dV (warps 0-3) and dK (warps 4-7) -> bf16 -------------------
+    if (ok) ok = mbar_wait_inl(bar_acc, 0, abort_sh, 90);
+    if (ok) {
+      tc_fence_after();
+      const uint32_t col = half ? C::COL_DK : C::COL_DV;
+      const float f = half ? a.scale : 1.0f;  // dK = scale dS^T Q: the MMAs used dS / scale
+      __nv_bfloat16* dst = (half ? a.dk : a.dv) + (static_cast<size_t>(bh_kv) * N + key) * C::D;
+#pragma unroll
+      for (int ch = 0; ch < C::D / 32; ++ch) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_base + col + ch * 32, v);
+        tmem_wait_ld();
+        if (key < N) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + ch * 32);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            d4[v4] = make_uint4(
+                pack_bf16x2(__uint_as_float(v[8 * v4 + 0]) * f, __uint_as_float(v[8 * v4 + 1]) * f),
+                pack_bf16x2(__uint_as_float(v[8 * v4 + 2]) * f, __uint_as_float(v[8 * v4 + 3]) * f),
+                pack_bf16x2(__uint_as_float(v[8 * v4 + 4]) * f, __uint_as_float(v[8 * v4 + 5]) * f),
+                pack_bf16x2(__uint_as_float(v[8 * v4 + 6]) * f, __uint_as_float(v[8 * v4 + 7]) * f));
+        }
+      }
+    }
+    tc_fence_before();
+    named_bar_sync_all(1, C::NTHREADS);
   }
 }
 

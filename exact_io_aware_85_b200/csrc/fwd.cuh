@@ -15,6 +15,8 @@
 //   warps 4-7  softmax for Q tile 1
 //   warp  8    TMA producer: Q0, Q1 once, then K_j and V_j through a ring
 //   warp  9    tcgen05.mma issuer (one thread) and TMEM owner
+//   warps 10-11 no role (they complete the third warpgroup, whose registers
+//              go to the softmax warpgroups)
 // Tensor memory (512 columns x 128 lanes, fp32):
 //   [0,128)   S0 = Q0 K_j^T   (P0 is written over its first columns as bf16)
 //   [128,256) S1 = Q1 K_j^T   (P1 likewise)
@@ -95,21 +97,18 @@ struct FwdCfg {
   // takes ~151 cycles per 16-deep step against ~108 from shared memory (at
   // N = 128, d = 128, tensor memory is the faster, ~73).
   static constexpr bool PV_SS = (EB == 2) && (D == 64) && !FP8P;
-  // Exponentials on the FMA pipe (exp2_fma2): this many of every 8 key pairs of
-  // a bf16 tile, the rest on the MUFU.  At d = 64 the MUFU is the busiest pipe
-  // (one exp per 128 FLOP of MMA against one per 256 at d = 128).
-#ifndef FA_EXP_POLY_D64
-#define FA_EXP_POLY_D64 0
-#endif
-#ifndef FA_EXP_POLY_D128
-#define FA_EXP_POLY_D128 0
-#endif
-  static constexpr int EXP_POLY = (EB == 2 && !FP8P) ? (D == 64 ? FA_EXP_POLY_D64 : FA_EXP_POLY_D128) : 0;
   static constexpr int P_BYTES = 128 * 128 * 2;  // one 128 x 128 bf16 P tile: two 64-key boxes
   static constexpr int OFF_P = OFF_V + NSTAGE * TILE_BYTES;
   static constexpr int SMEM_BYTES = OFF_P + (PV_SS ? 2 * P_BYTES : 0) + 1024;  // + alignment slack
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
-  static constexpr int NTHREADS = 320;
+  // Three warpgroups: two softmax warpgroups and one for the producer and MMA
+  // warps (two of its warps have no role).  Launched at 168 registers a thread
+  // (12 warps on 4 sub-partitions), the third warpgroup gives registers back and
+  // the softmax warpgroups take them: 8 x 32 x 216 + 4 x 32 x 72 = 64512 =
+  // 384 x 168, and 2 x 32 x 216 + 32 x 72 = 16128 <= 16384 per sub-partition.
+  static constexpr int NTHREADS = 384;
+  static constexpr int LAUNCH_REGS = 168, SOFTMAX_REGS = 216, OTHER_REGS = 72;
+  static_assert(8 * 32 * SOFTMAX_REGS + 4 * 32 * OTHER_REGS <= NTHREADS * LAUNCH_REGS, "register split");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
   static_assert(COL_O1 + D <= 512, "tensor memory budget");
 };
@@ -117,9 +116,9 @@ struct FwdCfg {
 // FP8P: P is cast to E4M3 before PV (bf16 operands); COUNT: FP8P that also
 // counts the P' values that flushed to zero.
 template <typename T, int D, bool FP8P, bool COUNT = false>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO, const FwdArgs a) {
   using C = FwdCfg<T, D, FP8P>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -182,12 +181,17 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
+  // Each warpgroup sets its register budget at the top of its own branch and the
+  // branches never rejoin: each ends at its own arrival on the teardown barrier.
+  if (warp >= 8) {
+  setmaxnreg_dec<C::OTHER_REGS>();
   if (warp == 8) {
     // ======================= TMA producer ===================================
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
+      if constexpr (C::EB == 2) tma_prefetch_desc(&tmO);
       mbar_arrive_expect_tx(&bar_q, (valid1 ? 2 : 1) * C::TILE_BYTES);
       for (int b = 0; b < C::NBOX; ++b) {
         tma_load_3d(smem + C::OFF_Q + b * C::BOX_BYTES, &tmQ, &bar_q, b * C::BOX_COLS, m0, bh);
@@ -360,7 +364,18 @@ __global__ void __launch_bounds__(320, 1)
       }
       __syncwarp();
     }
+  }
+  // teardown of the third warpgroup: once every warp has arrived, no MMA or TMEM
+  // access is in flight and warp 9 frees the tensor memory
+  tc_fence_before();
+  named_bar_sync_all(1, C::NTHREADS);
+  if (warp == 9) {
+    __syncwarp();  // reconverge after the barrier for the warp-wide dealloc
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
   } else {
+    setmaxnreg_inc<C::SOFTMAX_REGS>();
     // ======================= softmax warpgroups =============================
     const int i = warp >> 2;                       // Q tile
     const int r = threadIdx.x & 127;               // row in tile == TMEM lane
@@ -387,7 +402,7 @@ __global__ void __launch_bounds__(320, 1)
         const int j = rev ? n_steps - 1 - t : t;
         if (j >= kv_end) continue;
         const float c = C::EB == 1 ? c_base * a.sk[static_cast<size_t>(bh_k) * a.nqb + j] : c_base;
-        if (!(ok = mbar_wait(&bar_s[i], cnt & 1, &abort_sh, 10 + i))) break;
+        if (!(ok = mbar_wait_inl(&bar_s[i], cnt & 1, &abort_sh, 10 + i))) break;
         tc_fence_after();
         float sv[128];
         // first half of the row, then the second half streams in while the
@@ -485,15 +500,8 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
             for (int e = 0; e < PC; ++e) {
               const float2 x = ffma2(make_float2(sv[h * 2 * PC + 2 * e], sv[h * 2 * PC + 2 * e + 1]), c2, nm2);
-              float p0, p1;  // S p with FP8P, p otherwise
-              if ((e & 7) < C::EXP_POLY) {
-                const float2 pp = exp2_fma2(x);
-                p0 = pp.x;
-                p1 = pp.y;
-              } else {
-                p0 = ex2_approx(x.x);
-                p1 = ex2_approx(x.y);
-              }
+              const float p0 = ex2_approx(x.x);  // S p with FP8P, p otherwise
+              const float p1 = ex2_approx(x.y);
               rs4[e & 3] = fadd2(rs4[e & 3], make_float2(p0, p1));
               if constexpr (FP8P) {
                 uint32_t h2;
@@ -571,7 +579,7 @@ __global__ void __launch_bounds__(320, 1)
         ++cnt;
       }
       // ---- epilogue: O / l -> global, LSE -> global --------------------------
-      if (ok) ok = mbar_wait(&bar_o[i], 0, &abort_sh, 12 + i);
+      if (ok) ok = mbar_wait_inl(&bar_o[i], 0, &abort_sh, 12 + i);
       if (ok) {
         tc_fence_after();
         // l_run is the sum of S p when P is cast (S = 1 otherwise)
@@ -579,8 +587,33 @@ __global__ void __launch_bounds__(320, 1)
         // output: fp32 for fp32 inputs, bf16 otherwise (also for E4M3 operands)
         using OutT = typename std::conditional<C::EB == 4, float, __nv_bfloat16>::type;
         OutT* orow = reinterpret_cast<OutT*>(a.o) + (static_cast<size_t>(bh) * N + row) * D;
+        if constexpr (C::EB == 2) {
+          // bf16 operands: O goes through shared memory and leaves by TMA, whole
+          // rows at a time (rows past N are clipped by the tensor map).  The Q
+          // tile's buffer is free (every MMA that read it committed before
+          // bar_o) and has the O tile's size and 128-byte-swizzled layout:
+          // 16-byte chunk c of row r at r * 128 + ((c ^ r) & 7) * 16 in box c / 8.
+          uint8_t* ost = smem + C::OFF_Q + i * C::TILE_BYTES + r * 128;
 #pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t ov[32];
+            tmem_ld32(tO + ch * 32, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) {
+              const int c = ch * 4 + v4;  // 16-byte chunk of the row (8 columns)
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(ov[8 * v4 + 0]) * inv, __uint_as_float(ov[8 * v4 + 1]) * inv);
+              w.y = pack_bf16x2(__uint_as_float(ov[8 * v4 + 2]) * inv, __uint_as_float(ov[8 * v4 + 3]) * inv);
+              w.z = pack_bf16x2(__uint_as_float(ov[8 * v4 + 4]) * inv, __uint_as_float(ov[8 * v4 + 5]) * inv);
+              w.w = pack_bf16x2(__uint_as_float(ov[8 * v4 + 6]) * inv, __uint_as_float(ov[8 * v4 + 7]) * inv);
+              *reinterpret_cast<uint4*>(ost + (c >> 3) * C::BOX_BYTES + ((((c & 7) ^ r) & 7) << 4)) = w;
+            }
+          }
+          fence_proxy_async_smem();
+        }
+#pragma unroll
+        for (int ch = 0; ch < (C::EB == 2 ? 0 : D / 32); ++ch) {
           uint32_t ov[32];
           tmem_ld32(tO + ch * 32, ov);
           tmem_wait_ld();
@@ -608,6 +641,19 @@ __global__ void __launch_bounds__(320, 1)
         if (row < N)
           a.lse[static_cast<size_t>(bh) * N + row] = (m_run + log2f(l_run) - lg2S) * 0.69314718055994530942f;
       }
+      if constexpr (C::EB == 2) {
+        // every thread of the warpgroup arrives, also one whose wait gave up; the
+        // store goes out only if no wait of the CTA gave up before the barrier
+        named_bar_sync_all(2 + i, 128);  // the tile's 128 rows are in shared memory
+        if (r == 0 && ok && abort_sh == 0) {
+#pragma unroll
+          for (int b = 0; b < C::NBOX; ++b)
+            tma_store_3d(&tmO, smem + C::OFF_Q + i * C::TILE_BYTES + b * C::BOX_BYTES, b * C::BOX_COLS,
+                         m0 + 128 * i, bh);
+          tma_store_commit();
+          tma_store_wait_all();
+        }
+      }
       if constexpr (COUNT) {
         // flushed = admissible keys of the row minus those whose P' stayed non-zero
         uint32_t nk = 0;
@@ -626,14 +672,9 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
     }
-  }
-
-  // ---- teardown ------------------------------------------------------------
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 9) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    // teardown of the softmax warpgroups (see the third warpgroup's)
+    tc_fence_before();
+    named_bar_sync_all(1, C::NTHREADS);
   }
 }
 

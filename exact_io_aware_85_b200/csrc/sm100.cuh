@@ -90,6 +90,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   if (mbar_try_wait(a, parity)) return true;
   return mbar_wait_slow(a, parity, abort_flag, site);
 }
+// The same bounded wait with the slow path inlined, for warps whose register
+// budget was raised with setmaxnreg: ptxas cannot call an out-of-line function
+// from code that runs with more registers than the kernel was launched with.
+__device__ __forceinline__ bool mbar_wait_inl(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int site) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(a, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > FA_WAIT_LIMIT_NS) {
+        atomicCAS(&g_fa_status, 0, 5 /*FA_ERR_TIMEOUT*/ | (site << 8));
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
 
 // ----------------------------------------------------------------------------
 // TMA (tiled bulk tensor copies), global -> shared, completion on an mbarrier
@@ -102,12 +120,64 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
       : "memory");
 }
+// shared -> global tiled bulk store (rows past the tensor's extent are not
+// written); completion is tracked with the bulk-async group of the thread
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* smem_src, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(smem_src)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+// shared -> global tiled bulk reduction: the global tile += the shared tile
+// (element type of the tensor map), tracked like the stores
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, const void* smem_src, int x, int y, int z) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(smem_src)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void tma_store_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until every committed bulk store/reduction of this thread has finished
+// reading its shared-memory source (the global writes may still be in flight)
+__device__ __forceinline__ void tma_store_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// wait until every committed bulk store of this thread has completed
+__device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 // make generic-proxy shared-memory writes visible to the async proxy (TMA, tcgen05.mma)
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Named barrier that threads may reach from different code paths, also with
+// their warp diverged (the non-.aligned form counts arriving threads, wherever
+// and however they arrive).
+__device__ __forceinline__ void named_bar_sync_all(int id, int nthreads) {
+  asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Per-warpgroup register budgets (all four warps of a warpgroup execute the same
+// instruction).  `dec` returns registers to the block's pool, `inc` waits until
+// the pool holds enough; the pool is the block's launch allocation (threads x
+// registers per thread at launch), so the budgets must add up to no more.
+template <uint32_t R>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <uint32_t R>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
+}
+// from the launch budget FROM to TO, in whichever direction that is
+template <uint32_t FROM, uint32_t TO>
+__device__ __forceinline__ void setmaxnreg_to() {
+  if constexpr (TO > FROM)
+    setmaxnreg_inc<TO>();
+  else if constexpr (TO < FROM)
+    setmaxnreg_dec<TO>();
 }
 
 // ----------------------------------------------------------------------------
@@ -317,43 +387,6 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return d;
 }
-__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
-  float2 d;
-  asm("{\n\t.reg .b64 A, B, D;\n\t"
-      "mov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\t"
-      "sub.rn.f32x2 D, A, B;\n\tmov.b64 {%0, %1}, D;\n\t}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  return d;
-}
-
-// 2^x of two values on the FMA and integer pipes, so that part of a softmax
-// tile's exponentials run beside the MUFU ex2 instead of queueing for it.
-// x is clamped to >= -126 (exponent field >= 1 after the shift below), split as
-// x = j + f with j = round-to-nearest(x) (adding 1.5 * 2^23 leaves j in the low
-// mantissa bits; subtracting it again gives j exactly, and x - j is exact) and
-// |f| <= 1/2; 2^f comes from a degree-3 polynomial and j is added to the
-// exponent field as an integer.  The polynomial is the minimax approximation of
-// 2^f on [-1/2, 1/2] in relative error, found with the Remez exchange algorithm
-// (equioscillation at five points); with these float32 coefficients its largest
-// relative error is 7.5e-5, below the 2^-9 half-ulp of the bf16 P it feeds.
-// Inputs are <= 127 (the softmax arguments here are <= 8).
-__device__ __forceinline__ float2 exp2_fma2(float2 x) {
-  constexpr float c0 = 0.99992805719375610f, c1 = 0.69326096773147583f, c2 = 0.24261112511157990f,
-                  c3 = 0.05517166852951050f;
-  x.x = fmaxf(x.x, -126.f);
-  x.y = fmaxf(x.y, -126.f);
-  const float2 kRound = make_float2(12582912.f, 12582912.f);  // 1.5 * 2^23
-  const float2 t = fadd2(x, kRound);
-  const float2 f = fsub2(x, fsub2(t, kRound));
-  float2 p = ffma2(make_float2(c3, c3), f, make_float2(c2, c2));
-  p = ffma2(p, f, make_float2(c1, c1));
-  p = ffma2(p, f, make_float2(c0, c0));
-  // t's bits are 0x4B400000 + j: shifted left by 23 only j remains, in the exponent field
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
-}
-
 // three-input maximum (one instruction)
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
@@ -398,7 +431,9 @@ __device__ __forceinline__ uint32_t f16x2_sum_u32(uint32_t h2) {
 }
 
 // Wait used only on teardown paths: bounded by time, ignores the abort flag.
-__device__ __noinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+// Inlined: an out-of-line copy cannot be shared by warps whose register
+// budgets differ (setmaxnreg).
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   const uint32_t a = smem_u32(bar);
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(a, parity)) {
