@@ -38,10 +38,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # that kernel (dram__bytes_read.sum + dram__bytes_write.sum); reported only while
 # the kernel sources still hash to the values they were measured with.
 TRAFFIC = {
-    "prefill": {"bytes": 806519296 + 252521472, "src": ("fwd.cuh", "sm100.cuh"),
-                "sha1": "032a7705e1c46488fe7ced39baa01ab1630e52bc"},
-    "decode": {"bytes": 1073831168 + 3282688, "src": ("decode.cuh", "sm100.cuh"),
-               "sha1": "8dd9914892952b31c0692bb7e820ebf9d510d600"},
+    "prefill": {"bytes": 816854272 + 254902272, "src": ("fwd.cuh", "sm100.cuh"),
+                "sha1": "4d346ea54188e4429a60a810348ae4b3136888b0"},
+    "decode": {"bytes": 1073904896 + 3316224, "src": ("decode.cuh", "sm100.cuh"),
+               "sha1": "d0bcc3e7fb35ae74902bc06516df79ec510fb1bb"},
 }
 
 

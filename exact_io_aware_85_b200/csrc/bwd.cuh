@@ -915,12 +915,12 @@ __global__ void __launch_bounds__(448, 1)
 // pass.  dQ^T(t) is drained with coalesced fp32 reductions (a warp adds 32
 // consecutive head-dimension entries of one query row).
 // Warp roles (16 warps; registers per thread after setmaxnreg):
-//   warps 0-7   gradient warps (144): thread = key row (TMEM lane); warps 0-3
+//   warps 0-7   gradient warps (136): thread = key row (TMEM lane); warps 0-3
 //               queries 0-63 of the step, warps 4-7 queries 64-127
 //   warps 8-11  dQ drain and accumulator set-up (152): thread = TMEM lane
-//   warp  12    TMA producer, warp 13 MMA issuer and TMEM owner, 14-15 idle (72)
-// Launched at 128 registers a thread: 2 x 128 x 144 + 128 x 152 + 128 x 72 =
-// 65536 = 512 x 128, and 144 + 144 + 152 + 72 = 512 per sub-partition.
+//   warp  12    TMA producer, warp 13 MMA issuer and TMEM owner, 14-15 idle (88)
+// Launched at 128 registers a thread: 2 x 128 x 136 + 128 x 152 + 128 x 88 =
+// 65536 = 512 x 128, and 136 + 136 + 152 + 88 = 512 per sub-partition.
 struct BwdQ128Cfg {
   static constexpr int D = 128;
   static constexpr int BOX = 16384;             // 128 rows x 128 bytes
@@ -937,7 +937,7 @@ struct BwdQ128Cfg {
   static constexpr int SMEM_BYTES = OFF_BAR + 256;
   static constexpr uint32_t COL_DV = 0, COL_DK = 128, COL_S = 256, COL_DP = 384;
   static constexpr int NTHREADS = 512;
-  static constexpr int LAUNCH_REGS = 128, GRAD_REGS = 144, DRAIN_REGS = 152, OTHER_REGS = 72;
+  static constexpr int LAUNCH_REGS = 128, GRAD_REGS = 136, DRAIN_REGS = 152, OTHER_REGS = 88;
   static_assert(2 * 128 * GRAD_REGS + 128 * DRAIN_REGS + 128 * OTHER_REGS <= NTHREADS * LAUNCH_REGS,
                 "register split");
   static_assert(2 * GRAD_REGS + DRAIN_REGS + OTHER_REGS <= 512, "registers per sub-partition");
@@ -1050,6 +1050,11 @@ __global__ void __launch_bounds__(512, 1)
       const uint32_t k_addr = smem_u32(smem + C::OFF_K), v_addr = smem_u32(smem + C::OFF_V);
       const uint32_t q_addr = smem_u32(smem + C::OFF_Q), do_addr = smem_u32(smem + C::OFF_DO);
       const uint32_t ds_addr = smem_u32(smem + C::OFF_DS);
+      // base descriptors, built once; each MMA adds its K-step's byte offset
+      const uint64_t kd_k = make_sdesc_sw128(k_addr, 16, 1024);        // K, K-major (S^T)
+      const uint64_t vd_k = make_sdesc_sw128(v_addr, 16, 1024);        // V, K-major (dP^T)
+      const uint64_t kd_mn = make_sdesc_sw128(k_addr, C::BOX, 1024);   // K^T, MN-major (dQ^T)
+      const uint64_t dsd_mn = make_sdesc_sw128(ds_addr, C::BOX, 1024); // dS^T, MN-major (dQ^T)
       bool ok = mbar_wait_inl(bar_kv, 0, abort_sh, 81);
       for (int t = 0; ok && t < steps; ++t) {
         const int st = t % C::NST;
@@ -1057,6 +1062,8 @@ __global__ void __launch_bounds__(512, 1)
         if (!(ok = mbar_wait_inl(bar_ld_full + st, (t / C::NST) & 1, abort_sh, 82))) break;
         tc_fence_after();
         const uint32_t qa = q_addr + st * C::TILE, da = do_addr + st * C::TILE;
+        const uint64_t qd_k = make_sdesc_sw128(qa, 16, 1024), dod_k = make_sdesc_sw128(da, 16, 1024);
+        const uint64_t qd_mn = make_sdesc_sw128(qa, C::BOX, 1024), dod_mn = make_sdesc_sw128(da, C::BOX, 1024);
         // S^T = -LSE/scale + K_j Q_i^T (M = 128 keys, N = 128 queries, K = d), onto
         // the drain warps' fill of the columns that dV(t-1) read last
         if (!(ok = mbar_wait_inl(bar_s_init, ph, abort_sh, 91))) break;
@@ -1064,8 +1071,7 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t off = (k >> 2) * C::BOX + (k & 3) * 32;
-          mma_ss(tmem + C::COL_S, make_sdesc_sw128(k_addr + off, 16, 1024), make_sdesc_sw128(qa + off, 16, 1024),
-                 id_s, 1u);
+          mma_ss(tmem + C::COL_S, sdesc_add(kd_k, off), sdesc_add(qd_k, off), id_s, 1u);
         }
         mma_commit(bar_s_full);
         // dP^T = -D + V_j dO_i^T, onto the fill that replaced dQ^T(t-1)
@@ -1074,8 +1080,7 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t off = (k >> 2) * C::BOX + (k & 3) * 32;
-          mma_ss(tmem + C::COL_DP, make_sdesc_sw128(v_addr + off, 16, 1024), make_sdesc_sw128(da + off, 16, 1024),
-                 id_s, 1u);
+          mma_ss(tmem + C::COL_DP, sdesc_add(vd_k, off), sdesc_add(dod_k, off), id_s, 1u);
         }
         mma_commit(bar_dp_full);
         // dV += P^T dO_i (M = 128 keys, N = 128 columns, K = 128 queries): P^T in
@@ -1084,23 +1089,22 @@ __global__ void __launch_bounds__(512, 1)
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          mma_ts(tmem + C::COL_DV, tmem + C::COL_S + 64 * (k >> 2) + 8 * (k & 3),
-                 make_sdesc_sw128(da + k * 2048, C::BOX, 1024), id_g, (t > 0 || k > 0) ? 1u : 0u);
+          mma_ts(tmem + C::COL_DV, tmem + C::COL_S + 64 * (k >> 2) + 8 * (k & 3), sdesc_add(dod_mn, k * 2048), id_g,
+                 (t > 0 || k > 0) ? 1u : 0u);
         mma_commit(bar_s_free);  // P^T read: the S^T columns may be refilled
         // dK += dS^T Q_i (dS^T likewise over dP^T)
         if (!(ok = mbar_wait_inl(bar_ds_ready, ph, abort_sh, 85))) break;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + 64 * (k >> 2) + 8 * (k & 3),
-                 make_sdesc_sw128(qa + k * 2048, C::BOX, 1024), id_g, (t > 0 || k > 0) ? 1u : 0u);
+          mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + 64 * (k >> 2) + 8 * (k & 3), sdesc_add(qd_mn, k * 2048), id_g,
+                 (t > 0 || k > 0) ? 1u : 0u);
         mma_commit(bar_ld_empty + st);  // Q_i, dO_i, LSE_i, D_i read by everything that needs them
         // dQ_i^T = K_j^T dS^T (M = 128 columns, N = 128 queries, K = 128 keys) into
         // the dP^T columns, after dK has read dS^T there
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          mma_ss(tmem + C::COL_DP, make_sdesc_sw128(k_addr + k * 2048, C::BOX, 1024),
-                 make_sdesc_sw128(ds_addr + k * 2048, C::BOX, 1024), id_q, k > 0 ? 1u : 0u);
+          mma_ss(tmem + C::COL_DP, sdesc_add(kd_mn, k * 2048), sdesc_add(dsd_mn, k * 2048), id_q, k > 0 ? 1u : 0u);
         mma_commit(bar_dq_full);
       }
       if (ok) mma_commit(bar_acc);

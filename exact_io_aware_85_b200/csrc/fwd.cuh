@@ -225,13 +225,19 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp == 9) {
     // ======================= tcgen05.mma issuer =============================
-    // The whole warp follows the control flow (the fp32 path uses all lanes to
-    // round operand tiles); lane 0 alone issues MMAs and commits.
-    {
+    // Lane 0 alone issues MMAs and commits.  With fp32 operands the whole warp
+    // follows the control flow (all lanes round the operand tiles); otherwise the
+    // other lanes stay out of it: lanes spinning on the next barrier beside the
+    // issuing lane measurably slow its MMA issue.
+    constexpr bool kWarpWide = C::EB == 4;
+    if (kWarpWide || lane == 0) {
       const bool leader = lane == 0;
       // every lane waits (each gets the acquire), then the warp agrees on the outcome
       auto warp_wait = [&](uint64_t* bar, uint32_t parity, volatile int* ab, int site) {
-        return __all_sync(0xffffffffu, mbar_wait(bar, parity, ab, site));
+        if constexpr (kWarpWide)
+          return __all_sync(0xffffffffu, mbar_wait(bar, parity, ab, site));
+        else
+          return mbar_wait(bar, parity, ab, site);
       };
       constexpr uint32_t idesc_s = make_idesc(128, 128, ElemTraits<T>::kFmt, 0, 0);
       constexpr uint32_t idesc_pv = make_idesc(128, D, ElemTraits<T>::kFmt, 0, 1);
@@ -362,7 +368,7 @@ __global__ void __launch_bounds__(384, 1)
         mma_commit(&bar_done);
         mbar_wait_drain(&bar_done, 0, 100000000ull);
       }
-      __syncwarp();
+      if constexpr (kWarpWide) __syncwarp();
     }
   }
   // teardown of the third warpgroup: once every warp has arrived, no MMA or TMEM

@@ -232,6 +232,13 @@ __device__ __forceinline__ uint64_t make_sdesc_sw128(uint32_t smem_addr, uint32_
   return d;
 }
 
+// The descriptor of the same operand `bytes` further on: the start address is
+// the low 14-bit field (address >> 4), so the offset adds there directly as long
+// as address + bytes stays below 2^18 (all of shared memory does).  Building one
+// base descriptor per operand and adding constant offsets keeps the issuing
+// thread's work between MMAs to one add.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
+
 // Same, for the 128-byte swizzle with 32-byte atoms (layout type 1), the only
 // MN-major layout the tf32 MMA accepts; 4-row (512 B) swizzle period along K.
 __device__ __forceinline__ uint64_t make_sdesc_sw128_32b(uint32_t smem_addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
