@@ -38,6 +38,20 @@ __global__ void fa_watchdog_selftest_kernel(uint64_t limit_ns) {
   }
   __syncthreads();
 }
+// Self-test of the FMA-pipe exponential: y_fma = exp2_fma2(x), y_mufu = ex2.approx(x).
+__global__ void fa_exp2_selftest_kernel(const float* x, float* y_fma, float* y_mufu, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    const float2 p = exp2_fma2(make_float2(x[i], x[i + 1]));
+    y_fma[i] = p.x;
+    y_fma[i + 1] = p.y;
+    y_mufu[i] = ex2_approx(x[i]);
+    y_mufu[i + 1] = ex2_approx(x[i + 1]);
+  } else if (i < n) {
+    y_fma[i] = exp2_fma2(make_float2(x[i], 0.f)).x;
+    y_mufu[i] = ex2_approx(x[i]);
+  }
+}
 }  // namespace fa
 
 namespace {
@@ -607,6 +621,17 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
   if ((st = noalloc_scratch_for_current_device(&ws)) != FA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return launch_bwd_d(d, q, k, v, o, dO, lse, dq, dk, dv, B, H, N, causal, scale, ws, s);
+}
+
+int fa_exp2_selftest(const float* x, float* y_fma, float* y_mufu, int n, void* stream) {
+  if (!x || !y_fma || !y_mufu || n < 1) return FA_ERR_INVALID_ARG;
+  if (!aligned4(x) || !aligned4(y_fma) || !aligned4(y_mufu)) return FA_ERR_ALIGNMENT;
+  const int pairs = (n + 1) / 2;
+  fa::fa_exp2_selftest_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y_fma, y_mufu,
+                                                                                                  n);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return FA_OK;
 }
 
 int fa_watchdog_selftest(unsigned int limit_us, void* stream) {

@@ -97,6 +97,12 @@ struct FwdCfg {
   // takes ~151 cycles per 16-deep step against ~108 from shared memory (at
   // N = 128, d = 128, tensor memory is the faster, ~73).
   static constexpr bool PV_SS = (EB == 2) && (D == 64) && !FP8P;
+  // Exponentials on the FMA pipe (exp2_fma2) for 2 of every 8 key pairs of a
+  // bf16 tile at d = 64, the rest on the MUFU: there the MUFU is the busier pipe
+  // (one exponential per 128 FLOP of MMA against one per 256 at d = 128).
+  // Measured: 595 -> 616 TFLOP/s on the trading-day workload; 3 of 8 spill;
+  // at d = 128 any share is slower.
+  static constexpr int EXP_POLY = (EB == 2 && !FP8P && D == 64) ? 2 : 0;
   static constexpr int P_BYTES = 128 * 128 * 2;  // one 128 x 128 bf16 P tile: two 64-key boxes
   static constexpr int OFF_P = OFF_V + NSTAGE * TILE_BYTES;
   static constexpr int SMEM_BYTES = OFF_P + (PV_SS ? 2 * P_BYTES : 0) + 1024;  // + alignment slack
@@ -506,8 +512,15 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
             for (int e = 0; e < PC; ++e) {
               const float2 x = ffma2(make_float2(sv[h * 2 * PC + 2 * e], sv[h * 2 * PC + 2 * e + 1]), c2, nm2);
-              const float p0 = ex2_approx(x.x);  // S p with FP8P, p otherwise
-              const float p1 = ex2_approx(x.y);
+              float p0, p1;  // S p with FP8P, p otherwise
+              if ((e & 7) < C::EXP_POLY) {
+                const float2 pp = exp2_fma2(x);
+                p0 = pp.x;
+                p1 = pp.y;
+              } else {
+                p0 = ex2_approx(x.x);
+                p1 = ex2_approx(x.y);
+              }
               rs4[e & 3] = fadd2(rs4[e & 3], make_float2(p0, p1));
               if constexpr (FP8P) {
                 uint32_t h2;

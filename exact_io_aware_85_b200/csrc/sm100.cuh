@@ -394,6 +394,43 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return d;
 }
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 A, B, D;\n\t"
+      "mov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\t"
+      "sub.rn.f32x2 D, A, B;\n\tmov.b64 {%0, %1}, D;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// 2^x of two values on the FMA and integer pipes, so that part of a softmax
+// tile's exponentials run beside the MUFU ex2 instead of queueing for it.
+// x is clamped to >= -126 (exponent field >= 1 after the shift below), split as
+// x = j + f with j = round-to-nearest(x) (adding 1.5 * 2^23 leaves j in the low
+// mantissa bits; subtracting it again gives j exactly, and x - j is exact) and
+// |f| <= 1/2; 2^f comes from a degree-3 polynomial and j is added to the
+// exponent field as an integer.  The polynomial is the minimax approximation of
+// 2^f on [-1/2, 1/2] in relative error, found with the Remez exchange algorithm
+// (equioscillation at five points); with these float32 coefficients its largest
+// relative error is 7.5e-5, below the 2^-9 half-ulp of the bf16 P it feeds.
+// Inputs are <= 127 (the softmax arguments here are <= 8).
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  constexpr float c0 = 0.99992805719375610f, c1 = 0.69326096773147583f, c2 = 0.24261112511157990f,
+                  c3 = 0.05517166852951050f;
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 kRound = make_float2(12582912.f, 12582912.f);  // 1.5 * 2^23
+  const float2 t = fadd2(x, kRound);
+  const float2 f = fsub2(x, fsub2(t, kRound));
+  float2 p = ffma2(make_float2(c3, c3), f, make_float2(c2, c2));
+  p = ffma2(p, f, make_float2(c1, c1));
+  p = ffma2(p, f, make_float2(c0, c0));
+  // t's bits are 0x4B400000 + j: shifted left by 23 only j remains, in the exponent field
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
 // three-input maximum (one instruction)
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;

@@ -30,10 +30,11 @@ lib.fa_last_cuda_error.restype = _ci
 lib.fa_check_status.restype = _ci
 lib.fa_check_status.argtypes = [_vp]
 lib.fa_watchdog_selftest.argtypes = [ctypes.c_uint, _vp]
+lib.fa_exp2_selftest.argtypes = [_vp, _vp, _vp, _ci, _vp]
 
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_ALIGNMENT, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(6)
 EXPORTS = ("fa_fwd", "fa_fwd_f32", "fa_fwd_fp8p", "fa_bwd_workspace_bytes", "fa_bwd", "fa_status_string",
-           "fa_last_cuda_error", "fa_check_status", "fa_watchdog_selftest")
+           "fa_last_cuda_error", "fa_check_status", "fa_watchdog_selftest", "fa_exp2_selftest")
 
 
 class FAError(RuntimeError):
@@ -148,6 +149,15 @@ def fa_check_status(stream=None) -> int:
 def fa_last_cuda_error() -> int:
     """The cudaError_t of this host thread's last failed CUDA call inside the library."""
     return int(lib.fa_last_cuda_error())
+
+
+def fa_exp2_selftest(x, y_fma, y_mufu, stream=None) -> None:
+    """y_fma = the FMA-pipe exponential of the d = 64 softmax, y_mufu = ex2.approx,
+    both of the fp32 CUDA tensor x (same shape)."""
+    _need("fa_exp2_selftest", x=(x, torch.float32, None), y_fma=(y_fma, torch.float32, tuple(x.shape)),
+          y_mufu=(y_mufu, torch.float32, tuple(x.shape)))
+    _check(lib.fa_exp2_selftest(_ptr(x), _ptr(y_fma), _ptr(y_mufu), int(x.numel()), _stream(stream)),
+           "fa_exp2_selftest")
 
 
 def fa_watchdog_selftest(limit_us: int, stream=None) -> None:

@@ -201,6 +201,14 @@ int fa_last_cuda_error(void);
  * raised by work on another stream is reported too, once that work is done. */
 int fa_check_status(void* stream);
 
+/* Self-test of the exponential that part of the d = 64 softmax computes on the
+ * FMA pipe instead of the MUFU (range reduction x = j + f, |f| <= 1/2, then a
+ * degree-3 minimax polynomial for 2^f fitted by the Remez exchange algorithm):
+ * y_fma[i] = that exponential of x[i], y_mufu[i] = ex2.approx.ftz(x[i]), for
+ * n float32 values in device memory (4-byte aligned), x[i] <= 127.  Enqueued on
+ * `stream`.  Lets a test bound the polynomial's error against the hardware. */
+int fa_exp2_selftest(const float* x, float* y_fma, float* y_mufu, int n, void* stream);
+
 /* Failure-path self-test: launches a one-block kernel whose bounded wait on a
  * barrier that nothing signals gives up after limit_us microseconds (1 .. 10^7),
  * records FA_ERR_TIMEOUT in the device status word and returns; the CUDA context
