@@ -651,6 +651,7 @@ const char* fa_status_string(int status) {
     case FA_ERR_ALIGNMENT: return "FA_ERR_ALIGNMENT";
     case FA_ERR_CUDA: return "FA_ERR_CUDA";
     case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    case FA_ERR_CHECK: return "FA_ERR_CHECK";
     default: return "FA_ERR_UNKNOWN";
   }
 }

@@ -39,6 +39,30 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // is compiled as a single translation unit, so the definition lives here.
 __device__ int g_fa_status = 0;
 
+// Debug builds (-DFA_DEBUG) check the arguments of every TMA copy, tensor-memory
+// load/store and MMA before issuing it; a failed check records FA_ERR_CHECK (6)
+// with the check's site in bits 8-15 of the status word (the first failure
+// wins) and the operation is skipped, so a bad index is reported instead of
+// reaching the hardware.  Release builds compile the checks away.
+#ifdef FA_DEBUG
+__device__ __forceinline__ bool fa_check(bool ok, int site) {
+  if (!ok) atomicCAS(&g_fa_status, 0, 6 | (site << 8));
+  return ok;
+}
+#define FA_CHECK(cond, site) fa::fa_check((cond), (site))
+#else
+#define FA_CHECK(cond, site) true
+#endif
+// N of an instruction descriptor (bits 17-22 hold N / 8)
+__host__ __device__ constexpr uint32_t idesc_n(uint32_t idesc) { return ((idesc >> 17) & 63u) << 3; }
+// tensor memory: the columns [col, col + n) exist (512 allocated) and, for loads
+// and stores, the lanes are the calling warp's quarter (warp w reaches lanes
+// 32 (w % 4) .. 32 (w % 4) + 31)
+__device__ __forceinline__ bool tmem_cols_ok(uint32_t taddr, uint32_t n) { return (taddr & 0xFFFFu) + n <= 512u; }
+__device__ __forceinline__ bool tmem_quarter_ok(uint32_t taddr) {
+  return (taddr >> 21) == ((threadIdx.x >> 5) & 3u) && ((taddr >> 16) & 31u) == 0u;
+}
+
 // ----------------------------------------------------------------------------
 // mbarrier
 // ----------------------------------------------------------------------------
@@ -114,6 +138,9 @@ __device__ __forceinline__ bool mbar_wait_inl(uint64_t* bar, uint32_t parity, vo
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
                                             int z) {
+  // boxes land 128-byte aligned; x must start on a 16-byte boundary (every box
+  // here starts at a multiple of 8 elements of at most 2 bytes, or 32 fp32)
+  if (!FA_CHECK((smem_u32(smem_dst) & 127u) == 0 && x >= 0 && (x & 7) == 0 && z >= 0, 200)) return;
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
@@ -123,6 +150,7 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
 // shared -> global tiled bulk store (rows past the tensor's extent are not
 // written); completion is tracked with the bulk-async group of the thread
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* smem_src, int x, int y, int z) {
+  if (!FA_CHECK((smem_u32(smem_src) & 127u) == 0 && x >= 0 && (x & 7) == 0 && y >= 0 && z >= 0, 201)) return;
   asm volatile(
       "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
           reinterpret_cast<uint64_t>(map)),
@@ -132,6 +160,7 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void*
 // shared -> global tiled bulk reduction: the global tile += the shared tile
 // (element type of the tensor map), tracked like the stores
 __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, const void* smem_src, int x, int y, int z) {
+  if (!FA_CHECK((smem_u32(smem_src) & 127u) == 0 && x >= 0 && (x & 7) == 0 && y >= 0 && z >= 0, 202)) return;
   asm volatile(
       "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
           reinterpret_cast<uint64_t>(map)),
@@ -253,6 +282,7 @@ __device__ __forceinline__ uint64_t make_sdesc_sw128_32b(uint32_t smem_addr, uin
 
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                        uint32_t accumulate) {
+  if (!FA_CHECK((d_tmem >> 16) == 0u && tmem_cols_ok(d_tmem, idesc_n(idesc)), 205)) return;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
@@ -262,6 +292,7 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t
 }
 __device__ __forceinline__ void mma_ss_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                             uint32_t accumulate) {
+  if (!FA_CHECK((d_tmem >> 16) == 0u && tmem_cols_ok(d_tmem, idesc_n(idesc)), 205)) return;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
@@ -272,6 +303,8 @@ __device__ __forceinline__ void mma_ss_tf32(uint32_t d_tmem, uint64_t adesc, uin
 // A operand from tensor memory (K-major, packed 2 x 16-bit per 32-bit column)
 __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                        uint32_t accumulate) {
+  if (!FA_CHECK((d_tmem >> 16) == 0u && tmem_cols_ok(d_tmem, idesc_n(idesc)) && (a_tmem >> 16) == 0u &&
+                    tmem_cols_ok(a_tmem, 8), 205)) return;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
@@ -281,6 +314,8 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
 }
 __device__ __forceinline__ void mma_ts_tf32(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                             uint32_t accumulate) {
+  if (!FA_CHECK((d_tmem >> 16) == 0u && tmem_cols_ok(d_tmem, idesc_n(idesc)) && (a_tmem >> 16) == 0u &&
+                    tmem_cols_ok(a_tmem, 8), 205)) return;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
@@ -291,6 +326,7 @@ __device__ __forceinline__ void mma_ts_tf32(uint32_t d_tmem, uint32_t a_tmem, ui
 // kind::f8f6f4 (E4M3 operands, K = 32 per instruction), A from shared memory or TMEM
 __device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                           uint32_t accumulate) {
+  if (!FA_CHECK((d_tmem >> 16) == 0u && tmem_cols_ok(d_tmem, idesc_n(idesc)), 205)) return;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
@@ -300,6 +336,8 @@ __device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t adesc, uint6
 }
 __device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                           uint32_t accumulate) {
+  if (!FA_CHECK((d_tmem >> 16) == 0u && tmem_cols_ok(d_tmem, idesc_n(idesc)) && (a_tmem >> 16) == 0u &&
+                    tmem_cols_ok(a_tmem, 8), 205)) return;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
@@ -322,6 +360,7 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  if (!FA_CHECK(tmem_quarter_ok(taddr) && tmem_cols_ok(taddr, 32), 203)) return;
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
       "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -333,6 +372,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  if (!FA_CHECK(tmem_quarter_ok(taddr) && tmem_cols_ok(taddr, 32), 204)) return;
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
       "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
@@ -344,12 +384,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  if (!FA_CHECK(tmem_quarter_ok(taddr) && tmem_cols_ok(taddr, 8), 204)) return;
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]), "r"(r[1]),
       "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
       : "memory");
 }
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  if (!FA_CHECK(tmem_quarter_ok(taddr) && tmem_cols_ok(taddr, 16), 204)) return;
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
       "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),

@@ -12,9 +12,12 @@ import os
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa.so")
+# FA_DEBUG=1 selects the build with device-side argument checks (FA_ERR_CHECK)
+_DEBUG = os.environ.get("FA_DEBUG") == "1"
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa_debug.so" if _DEBUG else "libfa.so")
 if not os.path.exists(_LIB_PATH):
-    raise ImportError(f"libfa.so is not built ({_LIB_PATH}); run `python -m exact_io_aware_85_b200.build`")
+    raise ImportError(f"{os.path.basename(_LIB_PATH)} is not built ({_LIB_PATH}); run "
+                      f"`python -m exact_io_aware_85_b200.build{' --debug' if _DEBUG else ''}`")
 
 lib = ctypes.CDLL(_LIB_PATH)
 _vp, _ci, _cf, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
@@ -32,7 +35,7 @@ lib.fa_check_status.argtypes = [_vp]
 lib.fa_watchdog_selftest.argtypes = [ctypes.c_uint, _vp]
 lib.fa_exp2_selftest.argtypes = [_vp, _vp, _vp, _ci, _vp]
 
-FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_ALIGNMENT, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(6)
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_ALIGNMENT, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_CHECK = range(7)
 EXPORTS = ("fa_fwd", "fa_fwd_f32", "fa_fwd_fp8p", "fa_bwd_workspace_bytes", "fa_bwd", "fa_status_string",
            "fa_last_cuda_error", "fa_check_status", "fa_watchdog_selftest", "fa_exp2_selftest")
 

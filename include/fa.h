@@ -61,7 +61,11 @@ typedef enum {
                              than FA_BWD_NOALLOC_MAX_BYTES (fa_bwd_noalloc) */
   FA_ERR_ALIGNMENT = 3,   /* a pointer without the alignment the conventions require */
   FA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed */
-  FA_ERR_TIMEOUT = 5      /* a device-side wait gave up (reported by fa_check_status) */
+  FA_ERR_TIMEOUT = 5,     /* a device-side wait gave up (reported by fa_check_status) */
+  FA_ERR_CHECK = 6        /* debug builds only (compiled with FA_DEBUG): a device-side
+                             argument check of a TMA copy, tensor-memory access or MMA
+                             failed and the operation was skipped (reported by
+                             fa_check_status; bits 8-15 of the raw word name the check) */
 } fa_status;
 
 /* Forward, bf16 in/out, fp32 accumulation on the tensor cores.
