@@ -284,6 +284,8 @@ def main():
     lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
     launches_per_step = 1
+    # A step is a function of a buffer set (the tensors its copies touch), so that
+    # the end-to-end leg can alternate two sets; everything else is shared.
     if w.backward:
         # training step: forward, then backward from the saved LSE (4 launches)
         g = torch.Generator(device="cuda")
@@ -292,23 +294,26 @@ def main():
         dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
         ws_buf = torch.empty(fa.fa_bwd_workspace_bytes(w.B, w.H, w.N, w.d), dtype=torch.uint8, device="cuda")
         launches_per_step = 4
+        inputs, outputs = ("q", "k", "v", "do"), ("dq", "dk", "dv", "lse")
 
-        def run():
-            fa.fa_fwd(q, k, v, o, lse, w.causal, w.scale)
-            fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, w.causal, w.scale, ws_buf)
+        def step(b):
+            fa.fa_fwd(b["q"], b["k"], b["v"], b["o"], b["lse"], w.causal, w.scale)
+            fa.fa_bwd(b["q"], b["k"], b["v"], b["o"], b["do"], b["lse"], b["dq"], b["dk"], b["dv"], w.causal, w.scale,
+                      ws_buf)
     elif w.sink:
         # FP8 P-cast, forward key order, S = 256, on sink inputs with Delta = 8
         k[..., :4, 0] = 8.0 * math.sqrt(w.d)
         k[..., 4:, 0] = 0.0
         q[..., 0] = 1.0
         stats = torch.zeros(4, dtype=torch.int64, device="cuda") if not w.variant else None
+        inputs, outputs = ("q", "k", "v"), ("o", "lse")
 
         if w.variant == "bf16":
-            def run():
-                fa.fa_fwd(q, k, v, o, lse, w.causal, w.scale)
+            def step(b):
+                fa.fa_fwd(b["q"], b["k"], b["v"], b["o"], b["lse"], w.causal, w.scale)
         else:
-            def run():
-                fa.fa_fwd_fp8p(q, k, v, o, lse, w.causal, w.scale, 256.0, 0, stats, 4)
+            def step(b):
+                fa.fa_fwd_fp8p(b["q"], b["k"], b["v"], b["o"], b["lse"], w.causal, w.scale, 256.0, 0, stats, 4)
     elif w.dtype == "fp8":
         # E4M3 operands prepared once (quantisation with the random-sign Hadamard
         # rotation, outside the timed step); the step is the FP8 attention kernel
@@ -326,9 +331,13 @@ def main():
         qz1.record()
         torch.cuda.synchronize()
         quant_ms = qz0.elapsed_time(qz1)
+        inputs, outputs = ("q", "k", "v"), ("o", "lse")
 
-        def run():
-            fa.fa_fwd_fp8(q8, k8, v8, sq, sk, sv, o, lse, w.causal, w.scale, 256.0, 0)
+        def step(b):
+            fa.fa_fwd_fp8(q8, k8, v8, sq, sk, sv, b["o"], b["lse"], w.causal, w.scale, 256.0, 0)
+
+        def quantize(b):  # end to end: the fresh inputs are quantised inside the step
+            fa.fa_fp8_quantize(b["q"], b["k"], b["v"], signs, q8, k8, v8, sq, sk, sv)
     elif w.decode:
         # q, o: one row per head; k, v: the cache of H_kv heads
         q = q[:, :, 0].contiguous()
@@ -338,21 +347,33 @@ def main():
         v = v[:, : w.hkv].contiguous()
         ws_dec = torch.empty(fa.fa_decode_workspace_bytes(w.B, w.H, w.hkv, w.N, w.d), dtype=torch.uint8,
                              device="cuda")
+        inputs, outputs = ("q", "k", "v"), ("o", "lse")
 
-        def run():
-            fa.fa_decode(q, k, v, o, lse, w.scale, ws_dec)
+        def step(b):
+            fa.fa_decode(b["q"], b["k"], b["v"], b["o"], b["lse"], w.scale, ws_dec)
     elif w.hkv:
         k = k[:, : w.hkv].contiguous()
         v = v[:, : w.hkv].contiguous()
+        inputs, outputs = ("q", "k", "v"), ("o", "lse")
 
-        def run():
-            fa.fa_fwd_gqa(q, k, v, o, lse, w.causal, w.scale)
+        def step(b):
+            fa.fa_fwd_gqa(b["q"], b["k"], b["v"], b["o"], b["lse"], w.causal, w.scale)
     elif w.dtype == "bf16":
-        def run():
-            fa.fa_fwd(q, k, v, o, lse, w.causal, w.scale)
+        inputs, outputs = ("q", "k", "v"), ("o", "lse")
+
+        def step(b):
+            fa.fa_fwd(b["q"], b["k"], b["v"], b["o"], b["lse"], w.causal, w.scale)
     else:
-        def run():
-            fa.fa_fwd_f32(q, k, v, o, lse, w.causal, w.scale)
+        inputs, outputs = ("q", "k", "v"), ("o", "lse")
+
+        def step(b):
+            fa.fa_fwd_f32(b["q"], b["k"], b["v"], b["o"], b["lse"], w.causal, w.scale)
+    bufs = {"q": q, "k": k, "v": v, "o": o, "lse": lse}
+    if w.backward:
+        bufs.update(do=do, dq=dq, dk=dk, dv=dv)
+
+    def run():
+        step(bufs)
     small = 3 * q.numel() * q.element_size() < 126e6
     flush = torch.empty(int(256e6), dtype=torch.uint8, device="cuda") if small else None
 
@@ -392,49 +413,76 @@ def main():
     value = job_throughput(flops, step_ms, ws)
 
     # ---- end to end through the C ABI with pinned host buffers -----------------
-    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
-    ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-    hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
-    e2e_steps = max(3, min(args.steps, 10))
+    # Every step copies its inputs from pinned host memory, runs, and copies its
+    # results back.  Consecutive steps are pipelined over two device buffer sets
+    # and three streams (copies in, compute, copies out), so step i+1's inputs
+    # travel while step i computes and step i-1's results return; the same steps
+    # run back to back on one stream are reported too.
+    host_in = {n: bufs[n].cpu().pin_memory() for n in inputs}
+    host_out = [{n: torch.empty(bufs[n].shape, dtype=bufs[n].dtype, pin_memory=True) for n in outputs}
+                for _ in range(2)]
+    sets = [bufs, {n: (torch.empty_like(t) if n in inputs or n in outputs or n == "o" else t) for n, t in bufs.items()}]
+    e2e_steps = max(4, min(args.steps, 10))
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
 
-    if w.backward:
-        hdo = do.cpu().pin_memory()
-        hdq, hdk, hdv = (torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for _ in range(3))
+    def e2e_pipelined(n_steps, e_first=None, e_last=None):
+        if e_first is not None:
+            e_first.record(s_in)
+        for i in range(n_steps):
+            j = i % 2
+            b = sets[j]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_out[j])  # step i-2's results have left this set
+                for n in inputs:
+                    b[n].copy_(host_in[n], non_blocking=True)
+                ev_in[j].record(s_in)
+            stream.wait_event(ev_in[j])
+            if w.dtype == "fp8":
+                quantize(b)
+            step(b)
+            ev_comp[j].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_comp[j])
+                for n in outputs:
+                    host_out[j][n].copy_(b[n], non_blocking=True)
+                ev_out[j].record(s_out)
+        if e_last is not None:
+            e_last.record(s_out)
 
-    def e2e_step():
-        q.copy_(hq, non_blocking=True)
-        k.copy_(hk, non_blocking=True)
-        v.copy_(hv, non_blocking=True)
-        if w.backward:
-            do.copy_(hdo, non_blocking=True)
-        if w.dtype == "fp8":  # end to end includes the quantisation of the fresh inputs
-            fa.fa_fp8_quantize(q, k, v, signs, q8, k8, v8, sq, sk, sv)
-        run()
-        if w.backward:
-            hdq.copy_(dq, non_blocking=True)
-            hdk.copy_(dk, non_blocking=True)
-            hdv.copy_(dv, non_blocking=True)
-        else:
-            ho.copy_(o, non_blocking=True)
-        hl.copy_(lse, non_blocking=True)
+    def e2e_sequential_step():
+        for n in inputs:
+            bufs[n].copy_(host_in[n], non_blocking=True)
+        if w.dtype == "fp8":
+            quantize(bufs)
+        step(bufs)
+        for n in outputs:
+            host_out[0][n].copy_(bufs[n], non_blocking=True)
 
-    e2e_step()
+    e2e_pipelined(2)
+    e2e_sequential_step()
     torch.cuda.synchronize()
     barrier(ws)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     nvtx.range_push(f"fa_bench:{w.name}:e2e x{e2e_steps}")
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
+    e2e_pipelined(e2e_steps, e0, e1)
     torch.cuda.synchronize()
     nvtx.range_pop()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, ws)
-    h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
-    d2h = (3 * q.numel() * q.element_size() if w.backward else o.numel() * o.element_size()) + lse.numel() * 4
-    if w.backward:
-        h2d += do.numel() * do.element_size()
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_sequential_step()
+    s1.record(stream)
+    torch.cuda.synchronize()
+    seq_ms = max_over_ranks(s0.elapsed_time(s1) / e2e_steps, ws)
+    h2d = sum(bufs[n].numel() * bufs[n].element_size() for n in inputs)
+    d2h = sum(bufs[n].numel() * bufs[n].element_size() for n in outputs)
 
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     peak_note = f"{peak_src} bf16 burst (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback 1590 TFLOP/s"
@@ -515,7 +563,10 @@ def main():
                                        "mean": step_ms_local}},
             "clocks": clocks,
             "e2e": {"value": job_throughput(flops, e2e_ms, ws), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps,
+                    "how": "each step's inputs copied from pinned host memory and its results copied back; "
+                           "consecutive steps pipelined over two device buffer sets",
+                    "sequential": {"value": job_throughput(flops, seq_ms, ws), "ms_per_step": seq_ms}},
             "gpu_launches": args.steps * launches_per_step,
         }
         if w.dtype == "fp8":
