@@ -347,8 +347,10 @@ int noalloc_scratch_for_current_device(void** out) {
   return FA_OK;
 }
 // Head dim 256: one 128-row Q tile per CTA, 64-key K/V tiles (fwd256.cuh).
+template <bool FP8P, bool COUNT = false>
 int launch_fwd256(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv, int N,
-                  int causal, float scale, cudaStream_t stream) {
+                  int causal, float scale, cudaStream_t stream, float S = 1.f, int kv_order = 0,
+                  unsigned long long* stats = nullptr, int n_sink = 0) {
   using C = fa::Fwd256Cfg;
   const auto dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   CUtensorMap mq, mk, mv;
@@ -365,11 +367,15 @@ int launch_fwd256(const void* q, const void* k, const void* v, void* o, float* l
   a.group = H / Hkv;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.causal = causal ? 1 : 0;
-  cudaError_t e = cudaFuncSetAttribute(fa::fa_fwd256_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::SMEM_BYTES);
+  a.p_scale = S;
+  a.kv_order = kv_order;
+  a.stats = stats;
+  a.n_sink = n_sink;
+  auto kern = fa::fa_fwd256_kernel<FP8P, COUNT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_fail(e);
-  fa::fa_fwd256_kernel<<<static_cast<unsigned>(static_cast<long long>(a.nblk) * a.BH), C::NTHREADS, C::SMEM_BYTES,
-                         stream>>>(mq, mk, mv, a);
+  kern<<<static_cast<unsigned>(static_cast<long long>(a.nblk) * a.BH), C::NTHREADS, C::SMEM_BYTES, stream>>>(mq, mk,
+                                                                                                          mv, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return FA_OK;
@@ -410,7 +416,7 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   int st = check_common(q, k, v, o, lse, B, H, N, d, scale, true);
   if (st != FA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d == 256) return launch_fwd256(q, k, v, o, lse, B, H, H, N, causal, scale, s);
+  if (d == 256) return launch_fwd256<false>(q, k, v, o, lse, B, H, H, N, causal, scale, s);
   if (d == 64) return launch_fwd<__nv_bfloat16, 64, false>(q, k, v, o, lse, B, H, N, causal, scale, 1.f, 0, nullptr, 0, s);
   return launch_fwd<__nv_bfloat16, 128, false>(q, k, v, o, lse, B, H, N, causal, scale, 1.f, 0, nullptr, 0, s);
 }
@@ -427,13 +433,16 @@ int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* 
 int fa_fwd_fp8p(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
                 int causal, float scale, float S, int kv_order, unsigned long long* stats, int n_sink,
                 void* stream) {
-  int st = check_common(q, k, v, o, lse, B, H, N, d, scale);
+  int st = check_common(q, k, v, o, lse, B, H, N, d, scale, true);
   if (st != FA_OK) return st;
   if (!(std::isfinite(S) && S > 0.f)) return FA_ERR_INVALID_ARG;
   if (kv_order != 0 && kv_order != 1) return FA_ERR_INVALID_ARG;
   if (n_sink < 0) return FA_ERR_INVALID_ARG;
   if (stats && (reinterpret_cast<uintptr_t>(stats) & 7u)) return FA_ERR_ALIGNMENT;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 256)  // 64-key tiles: the running max of the P-cast moves once per 64 keys
+    return stats ? launch_fwd256<true, true>(q, k, v, o, lse, B, H, H, N, causal, scale, s, S, kv_order, stats, n_sink)
+                 : launch_fwd256<true>(q, k, v, o, lse, B, H, H, N, causal, scale, s, S, kv_order, nullptr, n_sink);
   // the flush counting is a separate instantiation: without stats the kernel carries none of it
   if (d == 64)
     return stats ? launch_fwd<__nv_bfloat16, 64, true, true>(q, k, v, o, lse, B, H, N, causal, scale, S, kv_order,
@@ -452,7 +461,7 @@ int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
   if (st != FA_OK) return st;
   if (H_kv < 1 || H % H_kv != 0) return FA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d == 256) return launch_fwd256(q, k, v, o, lse, B, H, H_kv, N, causal, scale, s);
+  if (d == 256) return launch_fwd256<false>(q, k, v, o, lse, B, H, H_kv, N, causal, scale, s);
   if (d == 64)
     return launch_fwd<__nv_bfloat16, 64, false>(q, k, v, o, lse, B, H, N, causal, scale, 1.f, 0, nullptr, 0, s,
                                                 nullptr, nullptr, nullptr, H_kv);
@@ -534,10 +543,12 @@ int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, 
   return FA_OK;
 }
 
-int fa_fp8_quantize(const void* q, const void* k, const void* v, const float* signs, void* q8, void* k8, void* v8,
-                    float* sq, float* sk, float* sv, int B, int H, int N, int d, void* stream) {
+int fa_fp8_quantize_gqa(const void* q, const void* k, const void* v, const float* signs, void* q8, void* k8,
+                        void* v8, float* sq, float* sk, float* sv, int B, int H, int H_kv, int N, int d,
+                        void* stream) {
   if (!q || !k || !v || !q8 || !k8 || !v8 || !sq || !sk || !sv) return FA_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
+  if (H_kv < 1 || H % H_kv != 0) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (!sizes_fit(B, H, N, d)) return FA_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * H > 65535) return FA_ERR_UNSUPPORTED;  // heads are gridDim.y of the Q/K pass
@@ -547,7 +558,7 @@ int fa_fp8_quantize(const void* q, const void* k, const void* v, const float* si
        reinterpret_cast<uintptr_t>(signs)) & 3u)
     return FA_ERR_ALIGNMENT;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int BH = B * H;
+  const int BH = B * H, BHkv = B * H_kv;
   fa::Fp8QuantArgs a;
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.k = static_cast<const __nv_bfloat16*>(k);
@@ -561,9 +572,11 @@ int fa_fp8_quantize(const void* q, const void* k, const void* v, const float* si
   a.sv = sv;
   a.N = N;
   a.nblk = (N + 127) / 128;
-  fa::fa_fp8_v_clear_kernel<<<(BH + 255) / 256, 256, 0, s>>>(sv, BH);
-  const dim3 grid(a.nblk, BH, 3);
-  const long long nvec = static_cast<long long>(BH) * N * (d / 8);
+  a.BH = BH;
+  a.BH_kv = BHkv;
+  fa::fa_fp8_v_clear_kernel<<<(BHkv + 255) / 256, 256, 0, s>>>(sv, BHkv);
+  const dim3 grid(a.nblk, BH, 3);  // BH >= BH_kv
+  const long long nvec = static_cast<long long>(BHkv) * N * (d / 8);
   if (d == 64) {
     fa::fa_fp8_qk_quant_kernel<64><<<grid, 128, 0, s>>>(a);
     fa::fa_fp8_v_quant_kernel<64><<<static_cast<unsigned>((nvec + 255) / 256), 256, 0, s>>>(a, nvec);
@@ -571,23 +584,35 @@ int fa_fp8_quantize(const void* q, const void* k, const void* v, const float* si
     fa::fa_fp8_qk_quant_kernel<128><<<grid, 128, 0, s>>>(a);
     fa::fa_fp8_v_quant_kernel<128><<<static_cast<unsigned>((nvec + 255) / 256), 256, 0, s>>>(a, nvec);
   }
-  fa::fa_fp8_v_scale_kernel<<<(BH + 255) / 256, 256, 0, s>>>(sv, BH);
+  fa::fa_fp8_v_scale_kernel<<<(BHkv + 255) / 256, 256, 0, s>>>(sv, BHkv);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return FA_OK;
 }
 
-int fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* sq, const float* sk, const float* sv,
-               void* o, float* lse, int B, int H, int N, int d, int causal, float scale, float S, int kv_order,
-               void* stream) {
+int fa_fp8_quantize(const void* q, const void* k, const void* v, const float* signs, void* q8, void* k8, void* v8,
+                    float* sq, float* sk, float* sv, int B, int H, int N, int d, void* stream) {
+  return fa_fp8_quantize_gqa(q, k, v, signs, q8, k8, v8, sq, sk, sv, B, H, H, N, d, stream);
+}
+
+int fa_fwd_fp8_gqa(const void* q8, const void* k8, const void* v8, const float* sq, const float* sk,
+                   const float* sv, void* o, float* lse, int B, int H, int H_kv, int N, int d, int causal, float scale,
+                   float S, int kv_order, void* stream) {
   int st = check_common(q8, k8, v8, o, lse, B, H, N, d, scale);
   if (st != FA_OK) return st;
   if (d != 128) return FA_ERR_UNSUPPORTED;  // E4M3 rows of 64 bytes would need the 64-byte swizzle
+  if (H_kv < 1 || H % H_kv != 0) return FA_ERR_INVALID_ARG;
   if (!sq || !sk || !sv) return FA_ERR_INVALID_ARG;
   if (!(std::isfinite(S) && S > 0.f)) return FA_ERR_INVALID_ARG;
   if (kv_order != 0 && kv_order != 1) return FA_ERR_INVALID_ARG;
   return launch_fwd<uint8_t, 128, true>(q8, k8, v8, o, lse, B, H, N, causal, scale, S, kv_order, nullptr, 0,
-                                        static_cast<cudaStream_t>(stream), sq, sk, sv);
+                                        static_cast<cudaStream_t>(stream), sq, sk, sv, H_kv);
+}
+
+int fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* sq, const float* sk, const float* sv,
+               void* o, float* lse, int B, int H, int N, int d, int causal, float scale, float S, int kv_order,
+               void* stream) {
+  return fa_fwd_fp8_gqa(q8, k8, v8, sq, sk, sv, o, lse, B, H, H, N, d, causal, scale, S, kv_order, stream);
 }
 
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {

@@ -65,9 +65,10 @@ struct Fp8QuantArgs {
   uint8_t* k8;
   uint8_t* v8;
   float* sq;           // [BH, nblk]
-  float* sk;           // [BH, nblk]
-  float* sv;           // [BH]: first the per-head amax (as ordered bits), then the scale
+  float* sk;           // [BH_kv, nblk]
+  float* sv;           // [BH_kv]: first the per-head amax (as ordered bits), then the scale
   int N, nblk;
+  int BH, BH_kv;       // query heads, key/value heads (B*H, B*H_kv)
 };
 
 // One CTA = one 128-row block of one (b,h); thread = row.
@@ -75,6 +76,8 @@ template <int D>
 __global__ void __launch_bounds__(128) fa_fp8_qk_quant_kernel(const Fp8QuantArgs a) {
   __shared__ float red[4];
   const int blk = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;  // 0 Q, 1 K, 2 V maxima
+  // grid.y covers the larger head count; the whole CTA leaves before any barrier
+  if (bh >= (which == 0 ? a.BH : a.BH_kv)) return;
   const int row = blk * 128 + threadIdx.x;
   const bool live = row < a.N;
   const __nv_bfloat16* src = which == 0 ? a.q : (which == 1 ? a.k : a.v);

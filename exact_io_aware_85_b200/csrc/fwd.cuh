@@ -71,7 +71,7 @@ struct FwdArgs {
   int n_sink;
   // full FP8 operands only: dequantisation scales of the E4M3 codes
   const float* sq;  // [BH, nqb] per 128-row block of Q
-  const float* sk;  // [BH, nqb] per 128-row block of K
+  const float* sk;  // [B*H_kv, nqb] per 128-row block of K
   const float* sv;  // [BH] per head of V
   int nqb;          // ceil(N / 128)
   int group;        // query heads per key/value head (1 = multi-head attention)

@@ -13,6 +13,9 @@
 // in order).  Because S(j+1) is issued before PV(j), "S(j+1) ready" does not
 // imply "PV(j) done": a softmax thread that must rescale O (the lazy correction
 // fires only when the row max grows by more than 2^8) first waits for PV(j).
+// FP8P: the E4M3 P-cast of "P-Cast precision in FP8 attention" on 64-key tiles
+// (the running max is exact, updated once per 64 keys, and the tiles can be
+// visited in reverse order); COUNT also counts the P' that flush to zero.
 #pragma once
 #include "sm100.cuh"
 
@@ -24,6 +27,10 @@ struct Fwd256Args {
   int N, BH, nblk, group;
   float scale_log2;
   int causal;
+  float p_scale;     // static scale S of the E4M3 P-cast (FP8P)
+  int kv_order;      // 0: key tiles 0..T-1, 1: T-1..0 (FP8P)
+  unsigned long long* stats;  // COUNT: [sink flushed, sink counted, non-sink flushed, non-sink counted]
+  int n_sink;
 };
 
 struct Fwd256Cfg {
@@ -42,6 +49,7 @@ struct Fwd256Cfg {
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
+template <bool FP8P, bool COUNT = false>
 __global__ void __launch_bounds__(192, 1)
     fa_fwd256_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const Fwd256Args a) {
@@ -66,6 +74,7 @@ __global__ void __launch_bounds__(192, 1)
   const int bh_kv = bh / a.group;
   const int n_kv = (N + 63) >> 6;
   const int T = a.causal ? min(n_kv, 2 * qt + 2) : n_kv;  // key tiles this Q tile sees
+  const bool rev = FP8P && a.kv_order;                       // visit them T-1 .. 0
 
   if (warp == 5) {
     tmem_alloc(&tmem_base_sh, 512);
@@ -105,13 +114,14 @@ __global__ void __launch_bounds__(192, 1)
         const int s = t & 1;
         const uint32_t ph = (t >> 1) & 1;
         if (!mbar_wait(&bar_ke[s], ph ^ 1, &abort_sh, 80)) break;
+        const int j = rev ? T - 1 - t : t;
         mbar_arrive_expect_tx(&bar_kf[s], C::KV_BYTES);
         for (int b = 0; b < 4; ++b)
-          tma_load_3d(smem + C::OFF_K + s * C::KV_BYTES + b * C::KV_BOX, &tmK, &bar_kf[s], b * 64, t * 64, bh_kv);
+          tma_load_3d(smem + C::OFF_K + s * C::KV_BYTES + b * C::KV_BOX, &tmK, &bar_kf[s], b * 64, j * 64, bh_kv);
         if (!mbar_wait(&bar_ve[s], ph ^ 1, &abort_sh, 81)) break;
         mbar_arrive_expect_tx(&bar_vf[s], C::KV_BYTES);
         for (int b = 0; b < 4; ++b)
-          tma_load_3d(smem + C::OFF_V + s * C::KV_BYTES + b * C::KV_BOX, &tmV, &bar_vf[s], b * 64, t * 64, bh_kv);
+          tma_load_3d(smem + C::OFF_V + s * C::KV_BYTES + b * C::KV_BOX, &tmV, &bar_vf[s], b * 64, j * 64, bh_kv);
       }
       mbar_wait_drain(&bar_q, 0, 100000000ull);
       for (int u = max(0, t - 2); u < t; ++u) {
@@ -174,10 +184,14 @@ __global__ void __launch_bounds__(192, 1)
     const int row = m0 + r;
     const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;
     const float c = a.scale_log2;
+    // with the P-cast the exponent carries log2(S): the exps give S p, l sums S p
+    const float lg2S = FP8P ? log2f(a.p_scale) : 0.f;
     float m_run = -INFINITY, l_run = 0.f;
+    uint32_t nf_sink = 0, nf_non = 0;  // COUNT: P' that did not flush, per key class
     bool ok = true;
     for (int t = 0; t < T && ok; ++t) {
       const int s = t & 1;
+      const int j = rev ? T - 1 - t : t;
       if (!(ok = mbar_wait(&bar_s[s], (t >> 1) & 1, &abort_sh, 87))) break;
       tc_fence_after();
       float sv[64];
@@ -185,7 +199,7 @@ __global__ void __launch_bounds__(192, 1)
       tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
       tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
       tmem_wait_ld();
-      const int kbase = t * 64;
+      const int kbase = j * 64;
       if (kbase + 64 > N || (a.causal && kbase + 63 > m0)) {
         const int lim = a.causal ? min(N - 1, row) : N - 1;
 #pragma unroll
@@ -201,22 +215,57 @@ __global__ void __launch_bounds__(192, 1)
         for (int u = 0; u < 8; ++u) mx8[u] = fmaxf(mx8[u], sv[e + u]);
       const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
       float m_new = fmaxf(m_run, mx * c);
-      if (m_new - m_run <= 8.0f) m_new = m_run;  // lazy correction (exps stay <= 2^8)
-      const float alpha = ex2_approx(m_run - m_new);
+      // lazy correction (exps stay <= 2^8); the P-cast needs the exact running max
+      if (!FP8P && m_new - m_run <= 8.0f) m_new = m_run;
+      // in reverse order a row can meet tiles that lie wholly past its diagonal
+      // before any admissible key: its max stays -inf, the tile adds nothing
+      const bool none_yet = FP8P && m_new == -INFINITY;
+      const float alpha = none_yet ? 1.f : ex2_approx(m_run - m_new);
       const bool rescale = t > 0 && __any_sync(0xffffffffu, m_new != m_run);
       l_run *= alpha;
       m_run = m_new;
-      const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_run, -m_run);
+      const float neg_m = lg2S - (none_yet ? 0.f : m_run);
+      const float2 c2 = make_float2(c, c), nm2 = make_float2(neg_m, neg_m);
+      // COUNT, tiles that hold sink keys: the P' of keys < n_sink that did not
+      // flush, counted apart with the same fma, ex2 and cast as the main pass
+      uint32_t nf_part = 0;
+      if constexpr (COUNT) {
+        if (kbase < a.n_sink && row < N) {
+#pragma unroll
+          for (int cc = 0; cc < 64; ++cc) {
+            if (kbase + cc < a.n_sink) {
+              const float qv = ex2_approx(fmaf(sv[cc], c, neg_m));
+              uint16_t e8;
+              asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(e8) : "f"(0.f), "f"(qv));
+              nf_part += (e8 & 0xFFu) ? 1u : 0u;
+            }
+          }
+        }
+      }
       float2 rs4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       uint32_t pk[32];
+      uint32_t nz2 = 0;  // COUNT: f16x2 counter of non-zero P' (at most 32 per half)
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
         const float2 x = ffma2(make_float2(sv[2 * e], sv[2 * e + 1]), c2, nm2);
-        const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
+        const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);  // S p with FP8P, p otherwise
         rs4[e & 3] = fadd2(rs4[e & 3], make_float2(p0, p1));
-        pk[e] = pack_bf16x2(p0, p1);
+        if constexpr (FP8P) {
+          uint32_t h2;
+          pk[e] = e4m3_round_bf16x2(p0, p1, h2);
+          if constexpr (COUNT) nz2 = count_nonzero_f16x2(h2, nz2);
+        } else {
+          pk[e] = pack_bf16x2(p0, p1);
+        }
       }
       tmem_st32(tS, pk);
+      if constexpr (COUNT) {
+        if (row < N) {
+          const uint32_t nf_tile = f16x2_sum_u32(nz2);
+          nf_sink += nf_part;
+          nf_non += nf_tile - nf_part;
+        }
+      }
       if (rescale) {
         // PV(t-1) may still be accumulating into O: wait for it before touching O
         if (!(ok = mbar_wait(&bar_pv, (t - 1) & 1, &abort_sh, 88))) break;
@@ -263,7 +312,25 @@ __global__ void __launch_bounds__(192, 1)
                                  pack_bf16x2(__uint_as_float(ov[8 * v4 + 6]) * inv, __uint_as_float(ov[8 * v4 + 7]) * inv));
         }
       }
-      if (row < N) a.lse[static_cast<size_t>(bh) * N + row] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
+      if (row < N)
+        a.lse[static_cast<size_t>(bh) * N + row] = (m_run + log2f(l_run) - lg2S) * 0.69314718055994530942f;
+    }
+    if constexpr (COUNT) {
+      // flushed = admissible keys of the row minus those whose P' stayed non-zero
+      uint32_t nk = 0;
+      if (row < N) nk = a.causal ? static_cast<uint32_t>(row + 1) : static_cast<uint32_t>(N);
+      const uint32_t ts = min(nk, static_cast<uint32_t>(max(a.n_sink, 0)));
+      const uint32_t tn = nk - ts;
+      const uint32_t v0 = __reduce_add_sync(0xffffffffu, ts - nf_sink);
+      const uint32_t v1 = __reduce_add_sync(0xffffffffu, ts);
+      const uint32_t v2 = __reduce_add_sync(0xffffffffu, tn - nf_non);
+      const uint32_t v3 = __reduce_add_sync(0xffffffffu, tn);
+      if (lane == 0) {
+        atomicAdd(a.stats + 0, static_cast<unsigned long long>(v0));
+        atomicAdd(a.stats + 1, static_cast<unsigned long long>(v1));
+        atomicAdd(a.stats + 2, static_cast<unsigned long long>(v2));
+        atomicAdd(a.stats + 3, static_cast<unsigned long long>(v3));
+      }
     }
   }
 

@@ -184,6 +184,8 @@ def fa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, causal: bool, scale: float, 
 
 lib.fa_fp8_quantize.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _vp]
 lib.fa_fwd_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _cf, _cf, _ci, _vp]
+lib.fa_fp8_quantize_gqa.argtypes = [_vp] * 10 + [_ci] * 5 + [_vp]
+lib.fa_fwd_fp8_gqa.argtypes = [_vp] * 8 + [_ci] * 6 + [_cf, _cf, _ci, _vp]
 
 
 def fa_fp8_quantize(q, k, v, signs, q8, k8, v8, sq, sk, sv, stream=None) -> None:
@@ -206,6 +208,31 @@ def fa_fwd_fp8(q8, k8, v8, sq, sk, sv, o, lse, causal: bool, scale: float, S: fl
           sk=(sk, _f32, (B, H, nb)), sv=(sv, _f32, (B, H)), o=(o, _bf, x), lse=(lse, _f32, (B, H, N)))
     _check(lib.fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq), _ptr(sk), _ptr(sv), _ptr(o), _ptr(lse), B, H, N,
                           d, int(causal), float(scale), float(S), int(kv_order), _stream(stream)), "fa_fwd_fp8")
+
+
+def fa_fp8_quantize_gqa(q, k, v, signs, q8, k8, v8, sq, sk, sv, stream=None) -> None:
+    """fa_fp8_quantize with k, v (and k8, v8, sk, sv) over H_kv key/value heads."""
+    B, H, N, d = _dims(q)
+    Hkv = int(k.shape[1]) if k.dim() == 4 else -1
+    x, xkv, nb = (B, H, N, d), (B, Hkv, N, d), (N + 127) // 128
+    _need("fa_fp8_quantize_gqa", q=(q, _bf, x), k=(k, _bf, xkv), v=(v, _bf, xkv),
+          signs=(signs, _f32, None if signs is None else (d,)), q8=(q8, _u8, x), k8=(k8, _u8, xkv),
+          v8=(v8, _u8, xkv), sq=(sq, _f32, (B, H, nb)), sk=(sk, _f32, (B, Hkv, nb)), sv=(sv, _f32, (B, Hkv)))
+    _check(lib.fa_fp8_quantize_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(signs), _ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq),
+                                   _ptr(sk), _ptr(sv), B, H, Hkv, N, d, _stream(stream)), "fa_fp8_quantize_gqa")
+
+
+def fa_fwd_fp8_gqa(q8, k8, v8, sq, sk, sv, o, lse, causal: bool, scale: float, S: float = 256.0, kv_order: int = 0,
+                   stream=None) -> None:
+    """fa_fwd_fp8 with k8, v8, sk, sv over H_kv key/value heads."""
+    B, H, N, d = _dims(q8)
+    Hkv = int(k8.shape[1]) if k8.dim() == 4 else -1
+    x, xkv, nb = (B, H, N, d), (B, Hkv, N, d), (N + 127) // 128
+    _need("fa_fwd_fp8_gqa", q8=(q8, _u8, x), k8=(k8, _u8, xkv), v8=(v8, _u8, xkv), sq=(sq, _f32, (B, H, nb)),
+          sk=(sk, _f32, (B, Hkv, nb)), sv=(sv, _f32, (B, Hkv)), o=(o, _bf, x), lse=(lse, _f32, (B, H, N)))
+    _check(lib.fa_fwd_fp8_gqa(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq), _ptr(sk), _ptr(sv), _ptr(o), _ptr(lse), B, H,
+                              Hkv, N, d, int(causal), float(scale), float(S), int(kv_order), _stream(stream)),
+           "fa_fwd_fp8_gqa")
 
 
 lib.fa_fwd_gqa.argtypes = [_vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _cf, _vp]

@@ -132,7 +132,9 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
  *            [0] sink P' that flushed to zero, [1] sink P counted,
  *            [2] non-sink P' that flushed to zero, [3] non-sink P counted,
  *            where a key is a sink when its index is < n_sink (n_sink >= 0).
- * q, k, v, o: bf16 [B,H,N,d]; lse: fp32 [B,H,N]. */
+ * Key tiles are 128 keys at d = 64 and 128 and 64 keys at d = 256: the running
+ * max moves once per tile, so the tile size is part of the result.
+ * q, k, v, o: bf16 [B,H,N,d]; lse: fp32 [B,H,N]; d in {64, 128, 256}. */
 int fa_fwd_fp8p(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
                 int causal, float scale, float S, int kv_order, unsigned long long* stats, int n_sink, void* stream);
 
@@ -189,6 +191,20 @@ int fa_fp8_quantize(const void* q, const void* k, const void* v, const float* si
 int fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* sq, const float* sk, const float* sv,
                void* o, float* lse, int B, int H, int N, int d, int causal, float scale, float S, int kv_order,
                void* stream);
+
+/* Grouped-query FP8 ("FlashAttention (IT)", "FlashAttention-2 (2023)": Multi-Query
+ * Attention, with the FP8 operands of "flash-attention-trading-models", "FA3"):
+ * k, v, k8, v8 [B,H_kv,N,d], sk [B,H_kv,ceil(N/128)], sv [B,H_kv]; q, q8, o
+ * [B,H,N,d], sq [B,H,ceil(N/128)], lse [B,H,N]; H a multiple of H_kv, query
+ * head h reads key/value head h / (H / H_kv).  Each key/value head is
+ * quantised once, so the codes and scales equal those fa_fp8_quantize gives
+ * for k, v repeated over the group.  Other conventions as fa_fp8_quantize and
+ * fa_fwd_fp8 (which are these calls with H_kv = H). */
+int fa_fp8_quantize_gqa(const void* q, const void* k, const void* v, const float* signs, void* q8, void* k8,
+                        void* v8, float* sq, float* sk, float* sv, int B, int H, int H_kv, int N, int d, void* stream);
+int fa_fwd_fp8_gqa(const void* q8, const void* k8, const void* v8, const float* sq, const float* sk,
+                   const float* sv, void* o, float* lse, int B, int H, int H_kv, int N, int d, int causal, float scale,
+                   float S, int kv_order, void* stream);
 
 /* Human-readable name of an fa_status code. */
 const char* fa_status_string(int status);

@@ -84,3 +84,25 @@ def test_sink_workload_full_size_against_closed_form():
         frac_r = st_r[2] / st_r[3]
         assert abs(frac_f - F) < 0.06, (delta, frac_f, F)
         assert frac_r <= 1.5 * max(frac_f, 1e-9) * 124 / (w.N - 4) + 1e-6, (delta, frac_r)
+
+
+@pytest.mark.parametrize("N,causal,delta,S,order", [(1000, False, 10.0, 256.0, 0), (1000, False, 7.0, 1.0, 1),
+                                                    (777, True, 8.0, 256.0, 1), (513, True, 0.0, 448.0, 0),
+                                                    (64, False, 12.0, 256.0, 1)])
+def test_fp8p_head_dim_256(N, causal, delta, S, order):
+    """d = 256: the P-cast on 64-key tiles (the emulation with B_c = 64), both key
+    orders; reverse order with the causal mask meets tiles wholly past a row's
+    diagonal before any admissible key."""
+    B, H, d = 1, 2, 256
+    x = synth.make_sink_inputs(B, H, N, d, delta, seed=33 + N)
+    o, lse, st = _run(x, B, H, N, d, causal, S, order)
+    o_em, lse_em, c_em = oracle.attn_fwd_fp8p(x["q"], x["k"], x["v"], causal, 1 / math.sqrt(d), S, order, 64, 4)
+    o_ex, lse_ex = oracle.attn_fwd(x["q"], x["k"], x["v"], causal, 1 / math.sqrt(d))
+    assert st[1] == c_em[1] and st[3] == c_em[3]
+    for a, b in ((st[0], c_em[0]), (st[2], c_em[2])):
+        assert abs(int(a) - int(b)) <= max(2, 1e-3 * max(int(b), 1))
+    assert np.isfinite(o).all() and np.abs(lse - lse_ex).max() <= 1e-3
+    mse_gpu = ((o - o_ex) ** 2).mean()
+    mse_em = ((o_em - o_ex) ** 2).mean()
+    assert abs(mse_gpu - mse_em) <= 0.1 * mse_em + 1e-7
+    _close_up_to_code_flips(o, o_em)
