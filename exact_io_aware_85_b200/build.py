@@ -13,7 +13,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libfa.so")
 LIB_DEBUG = os.path.join(PKG, "libfa_debug.so")
-SOURCES = ["api.cu", "sm100.cuh", "fwd.cuh", "bwd.cuh", "fp8.cuh", "decode.cuh", "fwd256.cuh"]
+SOURCES = ["api.cu", "sm100.cuh", "fwd.cuh", "bwd.cuh", "fp8.cuh", "decode.cuh", "fwd256.cuh", "bwd256.cuh"]
 HEADER = os.path.join(os.path.dirname(PKG), "include", "fa.h")
 
 

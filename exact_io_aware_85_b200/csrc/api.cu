@@ -19,6 +19,7 @@
 #include "fp8.cuh"
 #include "decode.cuh"
 #include "fwd256.cuh"
+#include "bwd256.cuh"
 
 namespace fa {
 // Self-test of the failure path: waits on an mbarrier that nothing will ever
@@ -186,6 +187,8 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   const int BH = B * H;
   const int BHkv = B * Hkv;
   const int n_tiles = (N + 127) / 128;
+  // d = 256 runs two CTAs per key tile
+  if (D == 256 && 2ll * n_tiles * BHkv >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
   const int npad = n_tiles * 128;
   float* lse2 = static_cast<float*>(workspace);
   float* dvec = lse2 + static_cast<size_t>(BH) * npad;
@@ -235,18 +238,18 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     if (fattr.numRegs < CQ::LAUNCH_REGS) return FA_ERR_UNSUPPORTED;
     kern<<<static_cast<unsigned>(static_cast<long long>(n_tiles) * BHkv), CQ::NTHREADS, CQ::SMEM_BYTES, stream>>>(
         mq, mk, mv, mdo, a);
-  } else if constexpr (D != 64) {
-    // 64-query variant: Q and dO tiles of 64 rows; at d = 256 two CTAs per key
-    // tile, one per 128-column slice of dV, dK and dQ
+  } else if constexpr (D == 256) {
+    // CTA pairs (clusters of 2) per key tile: rank 0 scores, dK and dQ[:, :128];
+    // rank 1 dP, dV and dQ[:, 128:]; P^T and dS^T exchanged in shared memory
     CUtensorMap mq64, mdo64;
     if ((st = encode_qkv_map(&mq64, q, dt, 2, D, N, BH, CU_TENSOR_MAP_SWIZZLE_128B, 64)) != FA_OK) return st;
     if ((st = encode_qkv_map(&mdo64, dO, dt, 2, D, N, BH, CU_TENSOR_MAP_SWIZZLE_128B, 64)) != FA_OK) return st;
-    using CQ = fa::BwdQ64Cfg<D>;
-    auto kern = fa::fa_bwd_main_q64_kernel<D>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, CQ::SMEM_BYTES);
+    using CP = fa::BwdPairCfg;
+    auto kern = fa::fa_bwd_main_pair256_kernel;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, CP::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e);
-    const dim3 grid(static_cast<unsigned>(static_cast<long long>(n_tiles) * BHkv), D / 128);
-    kern<<<grid, CQ::NTHREADS, CQ::SMEM_BYTES, stream>>>(mq64, mk, mv, mdo64, a);
+    kern<<<static_cast<unsigned>(2ll * n_tiles * BHkv), CP::NTHREADS, CP::SMEM_BYTES, stream>>>(mq64, mk, mv, mdo64,
+                                                                                              a);
   } else {
     using C = fa::BwdCfg<D>;
     auto kern = fa::fa_bwd_main_kernel<D>;

@@ -445,455 +445,6 @@ __global__ void __launch_bounds__(448, 1)
 }
 
 // ---------------------------------------------------------------------------
-// bwd_main, pipelined variant for d = 128 and 256 (64-query steps)
-// ---------------------------------------------------------------------------
-// Tensor memory at d = 128 cannot hold a second 128-query S^T tile, so this
-// variant walks the query tiles 64 at a time and double-buffers everything:
-//   TMEM: dV [0,128), dK [128,256), S^T buffers [256,320) [320,384),
-//         dP^T buffers [384,448) [448,512).  The gradient warps write P^T and
-//         dS^T (bf16, two per column) back over the start of each half's 32
-//         columns of S^T and dP^T, where dV += P^T dO and dK += dS^T Q read
-//         them as tensor-memory A operands; dQ^T of a step is then written
-//         over that step's S^T buffer.
-//   SMEM: K_j, V_j resident; Q_i, dO_i, LSE_i, D_i in three stages; dS^T
-//         (the B operand of dQ^T = K^T dS^T) double-buffered.
-// The MMA thread issues S^T(t+1) and dP^T(t+1) before it waits for the gradient
-// warps to finish step t, so the tensor core computes the next step's scores
-// while the current step's softmax gradient runs.  dQ is produced transposed,
-// dQ^T = K^T dS^T (M = d lanes, N = 64 queries), so the drain warps (thread =
-// head dimension) add into the fp32 accumulator with fully coalesced reductions.
-//
-// Head dimension 256 ("FlashAttention (IT)", section "FlashAttention-2 (2023)":
-// heads up to 256 wide) does not fit this tensor-memory budget whole: dV and dK
-// of a 128-key tile alone would take all 512 columns.  Each CTA therefore owns
-// one 128-wide slice of the head dimension (blockIdx.y): S^T and dP^T contract
-// over all 256 columns (recomputed by both CTAs of a key tile), while dV, dK and
-// dQ are produced for the CTA's slice only, since dV[:, h] = P^T dO[:, h],
-// dK[:, h] = dS^T Q[:, h] and dQ[:, h] = dS K[:, h].  K and V (64 KB each) stay
-// resident; Q and dO (32 KB each per 64 queries) leave room for one load stage,
-// filled in two halves with barriers of their own: the other slice's columns
-// (read by S^T and dP^T only) are refilled as soon as those two are done, while
-// the gradient and dV/dK/dQ of the step still run; this CTA's slice follows once
-// dK has finished with it.  The scores of the next step start on the early half.
-template <int DK>
-struct BwdQ64Cfg {
-  static_assert(DK == 128 || DK == 256, "head dimension");
-  static constexpr int D = 128;                 // output columns of dV, dK, dQ per CTA
-  static constexpr int NBOX = DK / 64;          // 128-byte swizzled column blocks of a row
-  static constexpr int KV_TILE = 128 * DK * 2;  // NBOX swizzled 16 KB blocks (128 rows)
-  static constexpr int Q_TILE = 64 * DK * 2;    // NBOX swizzled 8 KB blocks (64 rows)
-  static constexpr int KV_BOX = 16384, Q_BOX = 8192;
-  static constexpr int OP_TILE = 128 * 64 * 2;  // dS^T: 128 keys x 64 queries, one 16 KB block
-  static constexpr int OFF_K = 0;
-  static constexpr int OFF_V = OFF_K + KV_TILE;
-  static constexpr int NST = DK == 128 ? 3 : 1;   // Q/dO/LSE/D load stages
-  static constexpr int OFF_Q = OFF_V + KV_TILE;
-  static constexpr int OFF_DO = OFF_Q + NST * Q_TILE;
-  static constexpr int OFF_DS = OFF_DO + NST * Q_TILE;  // dS^T, 2 buffers (P^T stays in TMEM)
-  static constexpr int OFF_LSE = OFF_DS + 2 * OP_TILE;  // NST stages x 64 floats
-  static constexpr int OFF_DV = OFF_LSE + NST * 256;
-  static constexpr int OFF_BAR = OFF_DV + NST * 256;
-  static constexpr int SMEM_BYTES = OFF_BAR + 256;
-  static constexpr uint32_t COL_DV = 0, COL_DK = 128, COL_S = 256, COL_DP = 384;  // S, dP: +64 per buffer
-  static constexpr int NTHREADS = 448;
-  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-};
-
-template <int DK>
-__global__ void __launch_bounds__(448, 1)
-    fa_bwd_main_q64_kernel(const __grid_constant__ CUtensorMap tmQ64, const __grid_constant__ CUtensorMap tmK,
-                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO64,
-                           const BwdArgs a) {
-  using C = BwdQ64Cfg<DK>;
-  constexpr int D = C::D;
-  const int hd = blockIdx.y;  // 128-column slice of the head dimension produced here (0 when DK = 128)
-  extern __shared__ __align__(1024) uint8_t smem[];
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* bar_kv = bars + 0;
-  uint64_t* bar_ld_full = bars + 1;   // [NST]
-  uint64_t* bar_ld_empty = bars + 4;  // [NST]
-  uint64_t* bar_s_full = bars + 7;    // [2]
-  uint64_t* bar_dp_full = bars + 9;   // [2]
-  uint64_t* bar_pds = bars + 11;
-  uint64_t* bar_pds_free = bars + 12;  // [2]
-  uint64_t* bar_dq_full = bars + 14;   // [2]
-  uint64_t* bar_dq_free = bars + 16;   // [2]
-  uint64_t* bar_acc = bars + 18;
-  uint64_t* bar_done = bars + 19;
-  uint32_t* tmem_base_sh = reinterpret_cast<uint32_t*>(bars + 20);
-  volatile int* abort_sh = reinterpret_cast<volatile int*>(bars + 21);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int N = a.N;
-  const int bh_kv = blockIdx.x % a.BHkv;  // key/value head
-  const int j = blockIdx.x / a.BHkv;      // key tile of 128
-  const int n_q = (N + 63) >> 6;          // query tiles of 64
-  const int i0 = a.causal ? 2 * j : 0;
-  const int spq = n_q - i0;               // query tiles per query head
-  const int steps = spq * a.group;        // the walk covers every query head of the group
-  auto step_head = [&](int t) { return bh_kv * a.group + t / spq; };
-  auto step_tile = [&](int t) { return i0 + t % spq; };
-
-  if ((smem_u32(smem) & 1023u) != 0) {
-    if (threadIdx.x == 0) atomicCAS(&g_fa_status, 0, 4 /*FA_ERR_CUDA*/ | (98 << 8));
-    return;
-  }
-  if (warp == 13) {
-    tmem_alloc(tmem_base_sh, 512);
-    tmem_relinquish();
-  }
-  if (threadIdx.x == 0) {
-    *abort_sh = 0;
-    mbar_init(bar_kv, 1);
-    // DK = 256 fills its single stage in two halves, one slot each
-    for (int b = 0; b < (C::NST > 1 ? C::NST : 2); ++b) {
-      mbar_init(bar_ld_full + b, 1);
-      mbar_init(bar_ld_empty + b, 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar_s_full + b, 1);
-      mbar_init(bar_dp_full + b, 1);
-      mbar_init(bar_pds_free + b, 1);
-      mbar_init(bar_dq_full + b, 1);
-      mbar_init(bar_dq_free + b, 128);
-    }
-    mbar_init(bar_pds, 256);
-    mbar_init(bar_acc, 1);
-    mbar_init(bar_done, 1);
-    fence_mbar_init();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_base_sh;
-
-  if (warp == 12) {
-    // ============================ producer ===================================
-    if (lane == 0) {
-      tma_prefetch_desc(&tmQ64);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      tma_prefetch_desc(&tmDO64);
-      mbar_arrive_expect_tx(bar_kv, 2 * C::KV_TILE);
-      for (int b = 0; b < C::NBOX; ++b) {
-        tma_load_3d(smem + C::OFF_K + b * C::KV_BOX, &tmK, bar_kv, b * 64, j * 128, bh_kv);
-        tma_load_3d(smem + C::OFF_V + b * C::KV_BOX, &tmV, bar_kv, b * 64, j * 128, bh_kv);
-      }
-      int t = 0;
-      if constexpr (DK == 256) {
-        // one stage in two halves: slot 1 = the other slice's blocks, slot 0 =
-        // this CTA's slice plus the row statistics
-        const int ho = 1 - hd;
-        int n_early = 0;
-        for (; t < steps; ++t) {
-          const int i = step_tile(t), hq = step_head(t);
-          const uint32_t ph = t & 1;
-          if (!mbar_wait(bar_ld_empty + 1, ph ^ 1, abort_sh, 70)) break;
-          mbar_arrive_expect_tx(bar_ld_full + 1, 4 * C::Q_BOX);
-          for (int b = 2 * ho; b < 2 * ho + 2; ++b) {
-            tma_load_3d(smem + C::OFF_Q + b * C::Q_BOX, &tmQ64, bar_ld_full + 1, b * 64, i * 64, hq);
-            tma_load_3d(smem + C::OFF_DO + b * C::Q_BOX, &tmDO64, bar_ld_full + 1, b * 64, i * 64, hq);
-          }
-          n_early = t + 1;
-          if (!mbar_wait(bar_ld_empty, ph ^ 1, abort_sh, 60)) break;
-          mbar_arrive_expect_tx(bar_ld_full, 4 * C::Q_BOX + 512);
-          for (int b = 2 * hd; b < 2 * hd + 2; ++b) {
-            tma_load_3d(smem + C::OFF_Q + b * C::Q_BOX, &tmQ64, bar_ld_full, b * 64, i * 64, hq);
-            tma_load_3d(smem + C::OFF_DO + b * C::Q_BOX, &tmDO64, bar_ld_full, b * 64, i * 64, hq);
-          }
-          const size_t roff = static_cast<size_t>(hq) * a.Npad + static_cast<size_t>(i) * 64;
-          bulk_load(smem + C::OFF_LSE, a.lse2 + roff, 256, bar_ld_full);
-          bulk_load(smem + C::OFF_DV, a.dvec + roff, 256, bar_ld_full);
-        }
-        mbar_wait_drain(bar_kv, 0, 100000000ull);
-        if (n_early > 0) mbar_wait_drain(bar_ld_full + 1, (n_early - 1) & 1, 100000000ull);
-        if (t > 0) mbar_wait_drain(bar_ld_full, (t - 1) & 1, 100000000ull);
-      } else {
-        for (; t < steps; ++t) {
-          const int i = step_tile(t), hq = step_head(t);
-          const int s = t % C::NST;
-          const uint32_t ph = (t / C::NST) & 1;
-          if (!mbar_wait(bar_ld_empty + s, ph ^ 1, abort_sh, 60)) break;
-          mbar_arrive_expect_tx(bar_ld_full + s, 2 * C::Q_TILE + 512);
-          for (int b = 0; b < C::NBOX; ++b) {
-            tma_load_3d(smem + C::OFF_Q + s * C::Q_TILE + b * C::Q_BOX, &tmQ64, bar_ld_full + s, b * 64, i * 64, hq);
-            tma_load_3d(smem + C::OFF_DO + s * C::Q_TILE + b * C::Q_BOX, &tmDO64, bar_ld_full + s, b * 64, i * 64,
-                        hq);
-          }
-          const size_t roff = static_cast<size_t>(hq) * a.Npad + static_cast<size_t>(i) * 64;
-          bulk_load(smem + C::OFF_LSE + s * 256, a.lse2 + roff, 256, bar_ld_full + s);
-          bulk_load(smem + C::OFF_DV + s * 256, a.dvec + roff, 256, bar_ld_full + s);
-        }
-        mbar_wait_drain(bar_kv, 0, 100000000ull);
-        for (int u = max(0, t - C::NST); u < t; ++u)
-          mbar_wait_drain(bar_ld_full + u % C::NST, (u / C::NST) & 1, 100000000ull);
-      }
-    }
-  } else if (warp == 13) {
-    // ============================ MMA issuer =================================
-    if (lane == 0) {
-      constexpr uint32_t id_s = make_idesc(128, 64, kFmtBF16, 0, 0);    // S^T, dP^T: N = 64 queries
-      constexpr uint32_t id_g = make_idesc(128, D, kFmtBF16, 0, 1);     // dV, dK: A K-major, B MN-major
-      constexpr uint32_t id_q = make_idesc(128, 64, kFmtBF16, 1, 1);    // dQ^T: A = K^T, B = dS^T, both MN-major
-      const uint32_t k_addr = smem_u32(smem + C::OFF_K), v_addr = smem_u32(smem + C::OFF_V);
-      const uint32_t q_addr = smem_u32(smem + C::OFF_Q), do_addr = smem_u32(smem + C::OFF_DO);
-      const uint32_t ds_addr = smem_u32(smem + C::OFF_DS);
-      // dP^T(t) and S^T(t) at DK = 256: the other slice's half of Q_i and dO_i
-      // (slot 1) first, this CTA's slice (slot 0) last
-      auto phase_a2 = [&](int t) -> bool {
-        const int b = t & 1;
-        const int ho = 1 - hd;
-        auto dp_steps = [&](int h, bool first) {
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const int k = 8 * h + kk;
-            const uint32_t va = v_addr + (k >> 2) * C::KV_BOX + (k & 3) * 32;
-            const uint32_t db = do_addr + (k >> 2) * C::Q_BOX + (k & 3) * 32;
-            mma_ss(tmem + C::COL_DP + 64 * b, make_sdesc_sw128(va, 16, 1024), make_sdesc_sw128(db, 16, 1024), id_s,
-                   (first && kk == 0) ? 0u : 1u);
-          }
-        };
-        auto s_steps = [&](int h, bool first) {
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const int k = 8 * h + kk;
-            const uint32_t ka = k_addr + (k >> 2) * C::KV_BOX + (k & 3) * 32;
-            const uint32_t qb = q_addr + (k >> 2) * C::Q_BOX + (k & 3) * 32;
-            mma_ss(tmem + C::COL_S + 64 * b, make_sdesc_sw128(ka, 16, 1024), make_sdesc_sw128(qb, 16, 1024), id_s,
-                   (first && kk == 0) ? 0u : 1u);
-          }
-        };
-        if (!mbar_wait(bar_ld_full + 1, t & 1, abort_sh, 71)) return false;
-        tc_fence_after();
-        dp_steps(ho, true);
-        if (t >= 2) {
-          if (!mbar_wait(bar_dq_free + b, ((t - 2) >> 1) & 1, abort_sh, 63)) return false;
-          tc_fence_after();
-        }
-        s_steps(ho, true);
-        if (!mbar_wait(bar_ld_full, t & 1, abort_sh, 62)) return false;
-        tc_fence_after();
-        s_steps(hd, false);
-        mma_commit(bar_s_full + b);
-        dp_steps(hd, false);
-        mma_commit(bar_dp_full + b);
-        mma_commit(bar_ld_empty + 1);  // the other slice's half is read by nothing else
-        return true;
-      };
-      // dP^T(t) and S^T(t)
-      auto phase_a = [&](int t) -> bool {
-        if constexpr (DK == 256) return phase_a2(t);
-        const int b = t & 1;
-        const int st = t % C::NST;
-        if (!mbar_wait(bar_ld_full + st, (t / C::NST) & 1, abort_sh, 62)) return false;
-        tc_fence_after();
-        const uint32_t qa = q_addr + st * C::Q_TILE, da = do_addr + st * C::Q_TILE;
-        // dP^T = V_j dO_i^T first: its buffer was released when step t-2's
-        // gradient finished, so the tensor core has work while the dQ drain of
-        // step t-2 empties the S^T buffer
-#pragma unroll
-        for (int k = 0; k < DK / 16; ++k) {
-          const uint32_t va = v_addr + (k >> 2) * C::KV_BOX + (k & 3) * 32;
-          const uint32_t db = da + (k >> 2) * C::Q_BOX + (k & 3) * 32;
-          mma_ss(tmem + C::COL_DP + 64 * b, make_sdesc_sw128(va, 16, 1024), make_sdesc_sw128(db, 16, 1024), id_s,
-                 k > 0);
-        }
-        mma_commit(bar_dp_full + b);
-        if (t >= 2) {
-          if (!mbar_wait(bar_dq_free + b, ((t - 2) >> 1) & 1, abort_sh, 63)) return false;
-          tc_fence_after();
-        }
-        // S^T = K_j Q_i^T   (M = 128 keys, N = 64 queries, K = d), over dQ^T(t-2)
-#pragma unroll
-        for (int k = 0; k < DK / 16; ++k) {
-          const uint32_t ka = k_addr + (k >> 2) * C::KV_BOX + (k & 3) * 32;
-          const uint32_t qb = qa + (k >> 2) * C::Q_BOX + (k & 3) * 32;
-          mma_ss(tmem + C::COL_S + 64 * b, make_sdesc_sw128(ka, 16, 1024), make_sdesc_sw128(qb, 16, 1024), id_s,
-                 k > 0);
-        }
-        mma_commit(bar_s_full + b);
-        return true;
-      };
-      // dV(u), dK(u), dQ^T(u) once the gradient warps have written P^T and dS^T
-      auto phase_b = [&](int u) -> bool {
-        const int b = u & 1;
-        if (!mbar_wait(bar_pds, u & 1, abort_sh, 64)) return false;
-        tc_fence_after();
-        const int su = u % C::NST;
-        // this CTA's slice of the head dimension: blocks 2 hd and 2 hd + 1
-        const uint32_t qa = q_addr + su * C::Q_TILE + hd * 2 * C::Q_BOX;
-        const uint32_t da = do_addr + su * C::Q_TILE + hd * 2 * C::Q_BOX;
-        const uint32_t kh = k_addr + hd * 2 * C::KV_BOX;
-        const uint32_t dsa = ds_addr + b * C::OP_TILE;
-        // dV += P^T dO_i   (M = 128 keys, N = 128 columns, K = 64 queries; A = P^T in
-        // TMEM, each half's 32 queries packed at the start of its own 32 columns)
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          mma_ts(tmem + C::COL_DV, tmem + C::COL_S + 64 * b + (k >> 1) * 32 + (k & 1) * 8,
-                 make_sdesc_sw128(da + k * 2048, C::Q_BOX, 1024), id_g, (u > 0 || k > 0) ? 1u : 0u);
-        // dK += dS^T Q_i   (A = dS^T in TMEM, likewise over dP^T)
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + 64 * b + (k >> 1) * 32 + (k & 1) * 8,
-                 make_sdesc_sw128(qa + k * 2048, C::Q_BOX, 1024), id_g, (u > 0 || k > 0) ? 1u : 0u);
-        // dK was the stage's last reader (the gradient warps are done with its
-        // LSE and D): release it before dQ^T, which reads only K_j and dS^T
-        mma_commit(bar_ld_empty + su);
-        // dQ_i^T = K_j^T dS^T   (M = 128 columns, N = 64 queries, K = 128 keys), over S^T(u)
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          mma_ss(tmem + C::COL_S + 64 * b, make_sdesc_sw128(kh + k * 2048, C::KV_BOX, 1024),
-                 make_sdesc_sw128(dsa + k * 2048, C::KV_BOX, 1024), id_q, k > 0 ? 1u : 0u);
-        mma_commit(bar_dq_full + b);
-        mma_commit(bar_pds_free + b);
-        return true;
-      };
-      bool ok = mbar_wait(bar_kv, 0, abort_sh, 61);
-      for (int t = 0; ok && t <= steps; ++t) {
-        if constexpr (C::NST > 1) {
-          // the next step's scores are issued before this step's gradient is awaited
-          if (t < steps && !(ok = phase_a(t))) break;
-          if (t >= 1 && !(ok = phase_b(t - 1))) break;
-        } else {
-          // one load stage: Q_i and dO_i of step t arrive only after step t-1's
-          // last reader of the stage (dK) has been issued and has finished
-          if (t >= 1 && !(ok = phase_b(t - 1))) break;
-          if (t < steps && !(ok = phase_a(t))) break;
-        }
-      }
-      if (ok) mma_commit(bar_acc);
-      mma_commit(bar_done);
-      mbar_wait_drain(bar_done, 0, 100000000ull);
-    }
-  } else if (warp >= 8) {
-    // ============================ dQ drain ===================================
-    const int c = threadIdx.x - 256;  // head dimension == TMEM lane of dQ^T
-    const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-    for (int t = 0; t < steps; ++t) {
-      const int b = t & 1;
-      const int i = step_tile(t), hq = step_head(t);
-      if (!mbar_wait(bar_dq_full + b, (t >> 1) & 1, abort_sh, 65)) break;
-      tc_fence_after();
-      uint32_t v[64];
-      tmem_ld32(tmem + lane_base + C::COL_S + 64 * b, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-      tmem_ld32(tmem + lane_base + C::COL_S + 64 * b + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar_dq_free + b);  // the buffer is free as soon as it is in registers
-      float* dst = a.dq_acc + (static_cast<size_t>(hq) * a.Npad + static_cast<size_t>(i) * 64) * DK + hd * 128 + c;
-#pragma unroll
-      for (int q = 0; q < 64; ++q) atomicAdd(dst + static_cast<size_t>(q) * DK, __uint_as_float(v[q]));
-    }
-  } else {
-    // ============================ gradient warps =============================
-    const int half = warp >> 2;       // query columns [32 half, 32 half + 32) of each 64-query step
-    const int r = threadIdx.x & 127;  // key row in tile == TMEM lane
-    const int key = j * 128 + r;
-    const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-    const float cl = a.scale_log2;
-    bool ok = true;
-    for (int t = 0; t < steps && ok; ++t) {
-      const int i = step_tile(t);
-      const int b = t & 1;
-      const uint32_t ph = (t >> 1) & 1;
-      const int st = t % C::NST;
-      const float4* lse4 = reinterpret_cast<const float4*>(smem + C::OFF_LSE + st * 256) + half * 8;
-      const float4* dv4 = reinterpret_cast<const float4*>(smem + C::OFF_DV + st * 256) + half * 8;
-      const int q0 = i * 64 + half * 32;
-      const bool need_mask = (a.causal && q0 < j * 128 + 128) || key >= N;
-      if (!(ok = mbar_wait(bar_s_full + b, ph, abort_sh, 66))) break;
-      tc_fence_after();
-      float p[32];
-      tmem_ld32(tmem + lane_base + C::COL_S + 64 * b + half * 32, *reinterpret_cast<uint32_t(*)[32]>(&p[0]));
-      tmem_wait_ld();
-#pragma unroll
-      for (int e4 = 0; e4 < 8; ++e4) {
-        const float4 l4 = lse4[e4];
-        const float2 x01 = ffma2(make_float2(p[4 * e4], p[4 * e4 + 1]), make_float2(cl, cl), make_float2(-l4.x, -l4.y));
-        const float2 x23 = ffma2(make_float2(p[4 * e4 + 2], p[4 * e4 + 3]), make_float2(cl, cl), make_float2(-l4.z, -l4.w));
-        p[4 * e4] = ex2_approx(x01.x);
-        p[4 * e4 + 1] = ex2_approx(x01.y);
-        p[4 * e4 + 2] = ex2_approx(x23.x);
-        p[4 * e4 + 3] = ex2_approx(x23.y);
-      }
-      if (need_mask) {
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (key >= N || (a.causal && key > q0 + e)) p[e] = 0.f;
-      }
-      if (!(ok = mbar_wait(bar_dp_full + b, ph, abort_sh, 67))) break;
-      tc_fence_after();
-      uint32_t dp[32];
-      tmem_ld32(tmem + lane_base + C::COL_DP + 64 * b + half * 32, dp);
-      tmem_wait_ld();
-      uint32_t pw[16], dw[16];
-#pragma unroll
-      for (int e4 = 0; e4 < 8; ++e4) {
-        const float4 d4 = dv4[e4];
-        const float2 g01 = fmul2(make_float2(p[4 * e4], p[4 * e4 + 1]),
-                                 fadd2(make_float2(__uint_as_float(dp[4 * e4]), __uint_as_float(dp[4 * e4 + 1])),
-                                       make_float2(-d4.x, -d4.y)));
-        const float2 g23 = fmul2(make_float2(p[4 * e4 + 2], p[4 * e4 + 3]),
-                                 fadd2(make_float2(__uint_as_float(dp[4 * e4 + 2]), __uint_as_float(dp[4 * e4 + 3])),
-                                       make_float2(-d4.z, -d4.w)));
-        const float2 s01 = fmul2(g01, make_float2(a.scale, a.scale));
-        const float2 s23 = fmul2(g23, make_float2(a.scale, a.scale));
-        pw[2 * e4] = pack_bf16x2(p[4 * e4], p[4 * e4 + 1]);
-        pw[2 * e4 + 1] = pack_bf16x2(p[4 * e4 + 2], p[4 * e4 + 3]);
-        dw[2 * e4] = pack_bf16x2(s01.x, s01.y);
-        dw[2 * e4 + 1] = pack_bf16x2(s23.x, s23.y);
-      }
-      // P^T and dS^T (bf16, two per column) over the first 16 of this half's 32
-      // columns of the S^T and dP^T buffers, whose values are in registers now:
-      // the A operands of dV += P^T dO and dK += dS^T Q
-      tmem_st16(tmem + lane_base + C::COL_S + 64 * b + half * 32, pw);
-      tmem_st16(tmem + lane_base + C::COL_DP + 64 * b + half * 32, dw);
-      // dS^T once more in SMEM: the B operand of dQ^T = K^T dS^T
-      if (!(ok = mbar_wait(bar_pds_free + b, ph ^ 1, abort_sh, 68))) break;
-      uint8_t* db = smem + C::OFF_DS + b * C::OP_TILE;
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {  // 4 chunks of 8 queries: 16-byte chunk half*4 + cc of row r
-        const uint32_t off = sw128_off(r, half * 4 + cc);
-        *reinterpret_cast<uint4*>(db + off) = make_uint4(dw[4 * cc], dw[4 * cc + 1], dw[4 * cc + 2], dw[4 * cc + 3]);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      fence_proxy_async_smem();
-      mbar_arrive(bar_pds);
-    }
-    // ---- epilogue: dV (warps 0-3) and dK (warps 4-7) -> bf16 -------------------
-    if (ok) ok = mbar_wait(bar_acc, 0, abort_sh, 69);
-    if (ok) {
-      tc_fence_after();
-      const uint32_t col = half ? C::COL_DK : C::COL_DV;
-      __nv_bfloat16* dst = (half ? a.dk : a.dv) + (static_cast<size_t>(bh_kv) * N + key) * DK + hd * 128;
-#pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_base + col + ch * 32, v);
-        tmem_wait_ld();
-        if (key < N) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + ch * 32);
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            d4[v4] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * v4 + 0]), __uint_as_float(v[8 * v4 + 1])),
-                                pack_bf16x2(__uint_as_float(v[8 * v4 + 2]), __uint_as_float(v[8 * v4 + 3])),
-                                pack_bf16x2(__uint_as_float(v[8 * v4 + 4]), __uint_as_float(v[8 * v4 + 5])),
-                                pack_bf16x2(__uint_as_float(v[8 * v4 + 6]), __uint_as_float(v[8 * v4 + 7])));
-        }
-      }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 13) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
-  }
-}
-
-// ---------------------------------------------------------------------------
 // bwd_main at d = 128 with 128-query steps
 // ---------------------------------------------------------------------------
 // One CTA per (128-key tile, key/value head), K_j and V_j resident.  Each step

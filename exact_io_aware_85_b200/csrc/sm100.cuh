@@ -188,6 +188,89 @@ __device__ __forceinline__ void named_bar_sync_all(int id, int nthreads) {
   asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// ----------------------------------------------------------------------------
+// Thread-block clusters: two CTAs of one cluster exchange operand tiles through
+// distributed shared memory.  The copies are plain shared-to-shared bulk copies
+// into the peer CTA (no multicast loads); their completion is counted in bytes
+// on an mbarrier of the receiving CTA, like a TMA load's.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// every thread of every CTA of the cluster; release/acquire at cluster scope
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// the shared::cluster address of the same shared-memory object in CTA `rank`
+__device__ __forceinline__ uint32_t peer_smem(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+// one arrival on a barrier of the peer CTA that also raises its expected bytes
+__device__ __forceinline__ void mbar_arrive_expect_tx_peer(uint32_t peer_bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(peer_bar),
+               "r"(bytes)
+               : "memory");
+}
+// `bytes` (multiple of 16, both addresses 16-byte aligned) from this CTA's shared
+// memory into the peer's, completed on the peer's barrier `peer_bar`
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t peer_dst, const void* src, uint32_t bytes,
+                                                  uint32_t peer_bar) {
+  if (!FA_CHECK(((peer_dst | smem_u32(src) | bytes) & 15u) == 0, 206)) return;
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   peer_dst),
+               "r"(smem_u32(src)), "r"(bytes), "r"(peer_bar)
+               : "memory");
+}
+// 16 bytes into shared memory of a CTA of the cluster (a shared::cluster address)
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+// make this thread's generic-proxy writes to cluster shared memory visible to
+// the async proxy (the peer's tensor-core reads of them)
+__device__ __forceinline__ void fence_proxy_async_cluster() {
+  asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
+}
+// one arrival on a barrier of a CTA of the cluster, releasing this thread's
+// earlier writes at cluster scope
+__device__ __forceinline__ void mbar_arrive_peer(uint32_t peer_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(peer_bar) : "memory");
+}
+// Bounded wait as mbar_wait, acquiring at cluster scope: for barriers that the
+// peer CTA arrives on.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                  int site) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_cluster(a, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > FA_WAIT_LIMIT_NS) {
+        atomicCAS(&g_fa_status, 0, 5 /*FA_ERR_TIMEOUT*/ | (site << 8));
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
 // Per-warpgroup register budgets (all four warps of a warpgroup execute the same
 // instruction).  `dec` returns registers to the block's pool, `inc` waits until
 // the pool holds enough; the pool is the block's launch allocation (threads x
@@ -350,6 +433,15 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    smem_u32(bar))
                : "memory");
+}
+// The same arrival on the barrier at `bar`'s offset in each CTA of the cluster
+// named by `cta_mask` (bit r = cluster rank r); a signal only, no data moves.
+__device__ __forceinline__ void mma_commit_cluster(uint64_t* bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(cta_mask)
+      : "memory");
 }
 
 // ----------------------------------------------------------------------------

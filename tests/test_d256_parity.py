@@ -113,7 +113,7 @@ def test_d256_backward_long_sampled_heads():
 
 
 def test_d256_backward_deterministic_dk_dv():
-    # dK and dV of each 128-column slice accumulate inside one CTA in a fixed order
+    # dK (scores CTA) and dV (gradient CTA) each accumulate inside one CTA in a fixed order
     x = synth.make_inputs(1, 2, 384, 256, "bf16", seed=2400, with_grad=True)
     a = _bwd256(x, 1, 2, 2, 384, True)[2]
     b = _bwd256(x, 1, 2, 2, 384, True)[2]
