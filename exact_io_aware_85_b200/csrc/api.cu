@@ -82,13 +82,15 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // [B*H, N, d] row-major tensor seen as a 3-D TMA tensor (d, N, B*H); box of
 // 128 bytes x 128 rows with the 128-byte swizzle.  Rows beyond N read as zero.
 int encode_qkv_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, int d, int N, int BH,
-                   CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B, int box_rows = 128) {
+                   CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B, int box_rows = 128, int box_cols = 0) {
   auto fn = encode_fn();
   if (!fn) return cuda_fail(cudaErrorNotSupported);
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * elem_bytes,
                            static_cast<cuuint64_t>(d) * static_cast<cuuint64_t>(N) * elem_bytes};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem_bytes), static_cast<cuuint32_t>(box_rows), 1};
+  // boxes of 128-byte rows unless given (64-byte rows with the 64-byte swizzle)
+  if (box_cols <= 0) box_cols = 128 / elem_bytes;
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -135,11 +137,13 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   const int BH = B * H;
   CUtensorMap mq, mk, mv;
   int st;
-  if ((st = encode_qkv_map(&mq, q, dt, sizeof(T), D, N, BH)) != FA_OK) return st;
-  if ((st = encode_qkv_map(&mk, k, dt, sizeof(T), D, N, B * Hkv)) != FA_OK) return st;
+  // E4M3 rows at d = 64 are 64 bytes: whole-row boxes with the 64-byte swizzle
+  const CUtensorMapSwizzle swz = C::SW64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  if ((st = encode_qkv_map(&mq, q, dt, sizeof(T), D, N, BH, swz, 128, C::BOX_COLS)) != FA_OK) return st;
+  if ((st = encode_qkv_map(&mk, k, dt, sizeof(T), D, N, B * Hkv, swz, 128, C::BOX_COLS)) != FA_OK) return st;
   // fp32 V feeds the tf32 MMA as an MN-major operand, which needs the 32-byte-atom swizzle
   if ((st = encode_qkv_map(&mv, v, dt, sizeof(T), D, N, B * Hkv,
-                           sizeof(T) == 4 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
+                           sizeof(T) == 4 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : swz, 128, C::BOX_COLS)) != FA_OK)
     return st;
   // O leaves by TMA store when the operands are bf16 (the map is unused otherwise)
   CUtensorMap mo = mq;
@@ -603,13 +607,16 @@ int fa_fwd_fp8_gqa(const void* q8, const void* k8, const void* v8, const float* 
                    float S, int kv_order, void* stream) {
   int st = check_common(q8, k8, v8, o, lse, B, H, N, d, scale);
   if (st != FA_OK) return st;
-  if (d != 128) return FA_ERR_UNSUPPORTED;  // E4M3 rows of 64 bytes would need the 64-byte swizzle
   if (H_kv < 1 || H % H_kv != 0) return FA_ERR_INVALID_ARG;
   if (!sq || !sk || !sv) return FA_ERR_INVALID_ARG;
   if (!(std::isfinite(S) && S > 0.f)) return FA_ERR_INVALID_ARG;
   if (kv_order != 0 && kv_order != 1) return FA_ERR_INVALID_ARG;
-  return launch_fwd<uint8_t, 128, true>(q8, k8, v8, o, lse, B, H, N, causal, scale, S, kv_order, nullptr, 0,
-                                        static_cast<cudaStream_t>(stream), sq, sk, sv, H_kv);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 64)
+    return launch_fwd<uint8_t, 64, true>(q8, k8, v8, o, lse, B, H, N, causal, scale, S, kv_order, nullptr, 0, s, sq,
+                                         sk, sv, H_kv);
+  return launch_fwd<uint8_t, 128, true>(q8, k8, v8, o, lse, B, H, N, causal, scale, S, kv_order, nullptr, 0, s, sq, sk,
+                                        sv, H_kv);
 }
 
 int fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* sq, const float* sk, const float* sv,

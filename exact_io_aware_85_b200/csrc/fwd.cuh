@@ -80,9 +80,13 @@ struct FwdArgs {
 template <typename T, int D, bool FP8P>
 struct FwdCfg {
   static constexpr int EB = ElemTraits<T>::kBytes;
-  static constexpr int BOX_COLS = 128 / EB;            // elements in one 128-byte swizzled row
+  // swizzled row of a TMA box: 128 bytes, or 64 for E4M3 at d = 64 (a whole row,
+  // with the 64-byte swizzle)
+  static constexpr int ROW_BYTES = D * EB < 128 ? D * EB : 128;
+  static constexpr bool SW64 = ROW_BYTES == 64;
+  static constexpr int BOX_COLS = ROW_BYTES / EB;      // elements in one swizzled row
   static constexpr int NBOX = D / BOX_COLS;            // TMA boxes across the head dim
-  static constexpr int BOX_BYTES = 128 * 128;          // 128 rows x 128 bytes
+  static constexpr int BOX_BYTES = 128 * ROW_BYTES;    // 128 rows
   static constexpr int TILE_BYTES = NBOX * BOX_BYTES;  // one 128 x D tile
   static constexpr int KSTEP = 32 / EB;                // K elements per MMA (32 bytes)
   static constexpr int KSTEPS_PER_BOX = BOX_COLS / KSTEP;
@@ -121,6 +125,7 @@ struct FwdCfg {
   static_assert(8 * 32 * SOFTMAX_REGS + 4 * 32 * OTHER_REGS <= NTHREADS * LAUNCH_REGS, "register split");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
   static_assert(COL_O1 + D <= 512, "tensor memory budget");
+  static_assert(ROW_BYTES == 128 || (SW64 && EB == 1), "the 64-byte rows are E4M3 only");
 };
 
 // FP8P: P is cast to E4M3 before PV (bf16 operands); COUNT: FP8P that also
@@ -263,8 +268,9 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int k = 0; k < C::NK_QK; ++k) {
           const uint32_t off = (k / C::KSTEPS_PER_BOX) * C::BOX_BYTES + (k % C::KSTEPS_PER_BOX) * 32;
-          const uint64_t ad = make_sdesc_sw128(qa + off, 16, 1024);
-          const uint64_t bd = make_sdesc_sw128(ka + off, 16, 1024);
+          // K-major, 8-row groups 8 rows x ROW_BYTES apart
+          const uint64_t ad = C::SW64 ? make_sdesc_sw64(qa + off, 16, 512) : make_sdesc_sw128(qa + off, 16, 1024);
+          const uint64_t bd = C::SW64 ? make_sdesc_sw64(ka + off, 16, 512) : make_sdesc_sw128(ka + off, 16, 1024);
           if (!leader) continue;
           if constexpr (C::EB == 2)
             mma_ss(tmem + (i ? C::COL_S1 : C::COL_S0), ad, bd, idesc_s, k > 0);
@@ -282,10 +288,13 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t pa = smem_u32(smem + C::OFF_P) + i * C::P_BYTES;
 #pragma unroll
         for (int k = 0; k < C::NK_PV; ++k) {
-          // V is the MN-major B operand: 128B swizzle (bf16, E4M3) or the 32-byte-atom
-          // 128B swizzle (tf32, whose only MN-major layout), K rows 128 B apart.
-          const uint64_t bd = C::EB == 4 ? make_sdesc_sw128_32b(va + k * C::KSTEP * 128, C::BOX_BYTES, 512)
-                                         : make_sdesc_sw128(va + k * C::KSTEP * 128, C::BOX_BYTES, 1024);
+          // V is the MN-major B operand: 128B swizzle (bf16, E4M3), 64B swizzle (E4M3 at
+          // d = 64: N = 64 codes fill one row) or the 32-byte-atom 128B swizzle (tf32,
+          // whose only MN-major layout), K rows ROW_BYTES apart.
+          const uint32_t vk = va + k * C::KSTEP * C::ROW_BYTES;
+          const uint64_t bd = C::EB == 4 ? make_sdesc_sw128_32b(vk, C::BOX_BYTES, 512)
+                              : C::SW64  ? make_sdesc_sw64(vk, C::BOX_BYTES, 512)
+                                         : make_sdesc_sw128(vk, C::BOX_BYTES, 1024);
           const uint32_t acc = (pv_count[i] > 0 || k > 0) ? 1u : 0u;
           if (!leader) continue;
           if constexpr (C::PV_SS)

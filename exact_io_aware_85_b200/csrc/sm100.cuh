@@ -344,6 +344,18 @@ __device__ __forceinline__ uint64_t make_sdesc_sw128(uint32_t smem_addr, uint32_
   return d;
 }
 
+// The same for the 64-byte swizzle (layout type 4): rows of 64 bytes, the
+// pattern repeats every 8 rows (512 bytes).  Used for E4M3 tiles at d = 64.
+__device__ __forceinline__ uint64_t make_sdesc_sw64(uint32_t smem_addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;
+  d |= 4ull << 61;
+  return d;
+}
+
 // The descriptor of the same operand `bytes` further on: the start address is
 // the low 14-bit field (address >> 4), so the offset adds there directly as long
 // as address + bytes stays below 2^18 (all of shared memory does).  Building one

@@ -187,7 +187,8 @@ int fa_fp8_quantize(const void* q, const void* k, const void* v, const float* si
  * the kind::f8f6f4 tensor cores, the online softmax in fp32, P' = E4M3(S_p p)
  * (static scale S_p, key-tile order kv_order as in fa_fwd_fp8p), O += P' v8 on
  * the tensor cores, and O = acc * sv / (S_p * l) -> bf16 [B,H,N,d]; lse fp32
- * [B,H,N] of the quantised scores.  d = 128 only. */
+ * [B,H,N] of the quantised scores.  d in {64, 128} (64-byte E4M3 rows at d = 64
+ * are staged with the 64-byte swizzle). */
 int fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* sq, const float* sk, const float* sv,
                void* o, float* lse, int B, int H, int N, int d, int causal, float scale, float S, int kv_order,
                void* stream);

@@ -22,8 +22,8 @@ from helpers import to_dev
 
 pytestmark = pytest.mark.gpu
 
-CASES = [(1, 8, 2, 513, True, True, 0), (2, 4, 1, 300, False, True, 1), (1, 4, 4, 256, True, False, 0),
-         (1, 6, 3, 129, False, False, 1)]
+CASES = [(1, 8, 2, 513, True, True, 0, 128), (2, 4, 1, 300, False, True, 1, 128), (1, 4, 4, 256, True, False, 0, 128),
+         (1, 6, 3, 129, False, False, 1, 128), (1, 8, 2, 300, True, True, 1, 64)]
 
 
 def _quant(q, k, v, signs, gqa):
@@ -53,9 +53,9 @@ def _fwd(ops, causal, order, gqa):
     return o, lse
 
 
-@pytest.mark.parametrize("B,H,Hkv,N,causal,rotate,order", CASES)
-def test_fp8_gqa_matches_repeated_heads_and_emulation(B, H, Hkv, N, causal, rotate, order):
-    d, g = 128, H // Hkv
+@pytest.mark.parametrize("B,H,Hkv,N,causal,rotate,order,d", CASES)
+def test_fp8_gqa_matches_repeated_heads_and_emulation(B, H, Hkv, N, causal, rotate, order, d):
+    g = H // Hkv
     xq = synth.make_inputs(B, H, N, d, "bf16", seed=300 + N)
     xkv = synth.make_inputs(B, Hkv, N, d, "bf16", seed=400 + N)
     k_rep = np.repeat(xkv["k"], g, axis=1)

@@ -107,3 +107,20 @@ def test_incoherent_processing_lowers_gpu_error():
         err[rot] = float(np.sqrt(((o - o_ex) ** 2).mean()))
     ratio = err[False] / err[True]
     assert 2.0 <= ratio <= 3.5, (err, ratio)  # page: 2.6x lower than naive FP8
+
+
+@pytest.mark.parametrize("B,H,N,causal,rotate,order", [(1, 2, 1000, False, True, 0), (2, 1, 777, True, True, 1),
+                                                        (1, 2, 130, True, False, 0)])
+def test_fp8_forward_head_dim_64(B, H, N, causal, rotate, order):
+    """d = 64: 64-byte E4M3 rows, staged with the 64-byte swizzle."""
+    d = 64
+    x = synth.make_inputs(B, H, N, d, "bf16", seed=90 + N)
+    signs = synth.random_signs(d, seed=91) if rotate else None
+    o, lse = _fp8_forward(x, signs, causal, order)
+    o_em, lse_em = _oracle_fp8(x, signs, causal, order)
+    o_ex, _ = oracle.attn_fwd(x["q"], x["k"], x["v"], causal, 1 / math.sqrt(d))
+    assert np.abs(lse - lse_em).max() <= 2e-3
+    mse, mse_em = ((o - o_ex) ** 2).mean(), ((o_em - o_ex) ** 2).mean()
+    assert abs(mse - mse_em) <= 0.1 * mse_em
+    diff = np.abs(o - o_em)
+    assert (diff > 2e-2).mean() <= 1e-3 and diff.max() <= 0.15
