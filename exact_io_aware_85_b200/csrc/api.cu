@@ -353,21 +353,29 @@ int noalloc_scratch_for_current_device(void** out) {
   *out = g_noalloc_ptr[dev];
   return FA_OK;
 }
-// Head dim 256: one 128-row Q tile per CTA, 64-key K/V tiles (fwd256.cuh).
-template <bool FP8P, bool COUNT = false>
+// Head dim 256: one 128-row Q tile per CTA, 64-key K/V tiles (fwd256.cuh);
+// T = uint8_t takes E4M3 codes with their block scales.
+template <typename T, bool FP8P, bool COUNT = false>
 int launch_fwd256(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv, int N,
                   int causal, float scale, cudaStream_t stream, float S = 1.f, int kv_order = 0,
-                  unsigned long long* stats = nullptr, int n_sink = 0) {
-  using C = fa::Fwd256Cfg;
-  const auto dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+                  unsigned long long* stats = nullptr, int n_sink = 0, const float* sq = nullptr,
+                  const float* sk = nullptr, const float* sv = nullptr) {
+  using C = fa::Fwd256Cfg<sizeof(T)>;
+  const auto dt = sizeof(T) == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   CUtensorMap mq, mk, mv;
   int st;
-  if ((st = encode_qkv_map(&mq, q, dt, 2, 256, N, B * H, CU_TENSOR_MAP_SWIZZLE_128B, 128)) != FA_OK) return st;
-  if ((st = encode_qkv_map(&mk, k, dt, 2, 256, N, B * Hkv, CU_TENSOR_MAP_SWIZZLE_128B, 64)) != FA_OK) return st;
-  if ((st = encode_qkv_map(&mv, v, dt, 2, 256, N, B * Hkv, CU_TENSOR_MAP_SWIZZLE_128B, 64)) != FA_OK) return st;
+  if ((st = encode_qkv_map(&mq, q, dt, sizeof(T), 256, N, B * H, CU_TENSOR_MAP_SWIZZLE_128B, 128)) != FA_OK) return st;
+  if ((st = encode_qkv_map(&mk, k, dt, sizeof(T), 256, N, B * Hkv, CU_TENSOR_MAP_SWIZZLE_128B, 64)) != FA_OK)
+    return st;
+  if ((st = encode_qkv_map(&mv, v, dt, sizeof(T), 256, N, B * Hkv, CU_TENSOR_MAP_SWIZZLE_128B, 64)) != FA_OK)
+    return st;
   fa::Fwd256Args a;
   a.o = static_cast<__nv_bfloat16*>(o);
   a.lse = lse;
+  a.sq = sq;
+  a.sk = sk;
+  a.sv = sv;
+  a.nqb = (N + 127) / 128;
   a.N = N;
   a.BH = B * H;
   a.nblk = (N + 127) / 128;
@@ -378,7 +386,7 @@ int launch_fwd256(const void* q, const void* k, const void* v, void* o, float* l
   a.kv_order = kv_order;
   a.stats = stats;
   a.n_sink = n_sink;
-  auto kern = fa::fa_fwd256_kernel<FP8P, COUNT>;
+  auto kern = fa::fa_fwd256_kernel<T, FP8P, COUNT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_fail(e);
   kern<<<static_cast<unsigned>(static_cast<long long>(a.nblk) * a.BH), C::NTHREADS, C::SMEM_BYTES, stream>>>(mq, mk,
@@ -423,7 +431,7 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   int st = check_common(q, k, v, o, lse, B, H, N, d, scale, true);
   if (st != FA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d == 256) return launch_fwd256<false>(q, k, v, o, lse, B, H, H, N, causal, scale, s);
+  if (d == 256) return launch_fwd256<__nv_bfloat16, false>(q, k, v, o, lse, B, H, H, N, causal, scale, s);
   if (d == 64) return launch_fwd<__nv_bfloat16, 64, false>(q, k, v, o, lse, B, H, N, causal, scale, 1.f, 0, nullptr, 0, s);
   return launch_fwd<__nv_bfloat16, 128, false>(q, k, v, o, lse, B, H, N, causal, scale, 1.f, 0, nullptr, 0, s);
 }
@@ -448,8 +456,10 @@ int fa_fwd_fp8p(const void* q, const void* k, const void* v, void* o, float* lse
   if (stats && (reinterpret_cast<uintptr_t>(stats) & 7u)) return FA_ERR_ALIGNMENT;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 256)  // 64-key tiles: the running max of the P-cast moves once per 64 keys
-    return stats ? launch_fwd256<true, true>(q, k, v, o, lse, B, H, H, N, causal, scale, s, S, kv_order, stats, n_sink)
-                 : launch_fwd256<true>(q, k, v, o, lse, B, H, H, N, causal, scale, s, S, kv_order, nullptr, n_sink);
+    return stats ? launch_fwd256<__nv_bfloat16, true, true>(q, k, v, o, lse, B, H, H, N, causal, scale, s, S,
+                                                            kv_order, stats, n_sink)
+                 : launch_fwd256<__nv_bfloat16, true>(q, k, v, o, lse, B, H, H, N, causal, scale, s, S, kv_order,
+                                                      nullptr, n_sink);
   // the flush counting is a separate instantiation: without stats the kernel carries none of it
   if (d == 64)
     return stats ? launch_fwd<__nv_bfloat16, 64, true, true>(q, k, v, o, lse, B, H, N, causal, scale, S, kv_order,
@@ -468,7 +478,7 @@ int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
   if (st != FA_OK) return st;
   if (H_kv < 1 || H % H_kv != 0) return FA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d == 256) return launch_fwd256<false>(q, k, v, o, lse, B, H, H_kv, N, causal, scale, s);
+  if (d == 256) return launch_fwd256<__nv_bfloat16, false>(q, k, v, o, lse, B, H, H_kv, N, causal, scale, s);
   if (d == 64)
     return launch_fwd<__nv_bfloat16, 64, false>(q, k, v, o, lse, B, H, N, causal, scale, 1.f, 0, nullptr, 0, s,
                                                 nullptr, nullptr, nullptr, H_kv);
@@ -556,7 +566,7 @@ int fa_fp8_quantize_gqa(const void* q, const void* k, const void* v, const float
   if (!q || !k || !v || !q8 || !k8 || !v8 || !sq || !sk || !sv) return FA_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
   if (H_kv < 1 || H % H_kv != 0) return FA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
   if (!sizes_fit(B, H, N, d)) return FA_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * H > 65535) return FA_ERR_UNSUPPORTED;  // heads are gridDim.y of the Q/K pass
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q8) || !aligned16(k8) || !aligned16(v8))
@@ -587,6 +597,9 @@ int fa_fp8_quantize_gqa(const void* q, const void* k, const void* v, const float
   if (d == 64) {
     fa::fa_fp8_qk_quant_kernel<64><<<grid, 128, 0, s>>>(a);
     fa::fa_fp8_v_quant_kernel<64><<<static_cast<unsigned>((nvec + 255) / 256), 256, 0, s>>>(a, nvec);
+  } else if (d == 256) {
+    fa::fa_fp8_qk_quant_kernel<256><<<grid, 128, 0, s>>>(a);
+    fa::fa_fp8_v_quant_kernel<256><<<static_cast<unsigned>((nvec + 255) / 256), 256, 0, s>>>(a, nvec);
   } else {
     fa::fa_fp8_qk_quant_kernel<128><<<grid, 128, 0, s>>>(a);
     fa::fa_fp8_v_quant_kernel<128><<<static_cast<unsigned>((nvec + 255) / 256), 256, 0, s>>>(a, nvec);
@@ -605,13 +618,16 @@ int fa_fp8_quantize(const void* q, const void* k, const void* v, const float* si
 int fa_fwd_fp8_gqa(const void* q8, const void* k8, const void* v8, const float* sq, const float* sk,
                    const float* sv, void* o, float* lse, int B, int H, int H_kv, int N, int d, int causal, float scale,
                    float S, int kv_order, void* stream) {
-  int st = check_common(q8, k8, v8, o, lse, B, H, N, d, scale);
+  int st = check_common(q8, k8, v8, o, lse, B, H, N, d, scale, true);
   if (st != FA_OK) return st;
   if (H_kv < 1 || H % H_kv != 0) return FA_ERR_INVALID_ARG;
   if (!sq || !sk || !sv) return FA_ERR_INVALID_ARG;
   if (!(std::isfinite(S) && S > 0.f)) return FA_ERR_INVALID_ARG;
   if (kv_order != 0 && kv_order != 1) return FA_ERR_INVALID_ARG;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 256)
+    return launch_fwd256<uint8_t, true>(q8, k8, v8, o, lse, B, H, H_kv, N, causal, scale, s, S, kv_order, nullptr, 0,
+                                        sq, sk, sv);
   if (d == 64)
     return launch_fwd<uint8_t, 64, true>(q8, k8, v8, o, lse, B, H, N, causal, scale, S, kv_order, nullptr, 0, s, sq,
                                          sk, sv, H_kv);

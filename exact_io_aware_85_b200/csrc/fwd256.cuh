@@ -16,6 +16,9 @@
 // FP8P: the E4M3 P-cast of "P-Cast precision in FP8 attention" on 64-key tiles
 // (the running max is exact, updated once per 64 keys, and the tiles can be
 // visited in reverse order); COUNT also counts the P' that flush to zero.
+// Elem = uint8_t: E4M3 operands with block scales ("flash-attention-trading-models",
+// "FA3" item 3) on kind::f8f6f4 MMAs: rows of 256 bytes in two 128-byte boxes,
+// 32 keys per PV step, P cast to E4M3 codes (four per tensor-memory column).
 #pragma once
 #include "sm100.cuh"
 
@@ -24,6 +27,10 @@ namespace fa {
 struct Fwd256Args {
   __nv_bfloat16* o;
   float* lse;
+  const float* sq;  // E4M3: [BH, nqb] scale per 128-row block of Q
+  const float* sk;  // E4M3: [B*H_kv, nqb] per 128-row block of K
+  const float* sv;  // E4M3: [B*H_kv] per head of V
+  int nqb;          // ceil(N / 128)
   int N, BH, nblk, group;
   float scale_log2;
   int causal;
@@ -33,13 +40,19 @@ struct Fwd256Args {
   int n_sink;
 };
 
+template <int EB>
 struct Fwd256Cfg {
   static constexpr int D = 256;
   static constexpr int BM = 128, BN = 64;
-  static constexpr int Q_BOX = 128 * 128;   // 128 rows x 128 B (64 columns)
-  static constexpr int KV_BOX = 64 * 128;   // 64 rows x 128 B
-  static constexpr int Q_BYTES = 4 * Q_BOX;     // 64 KB
-  static constexpr int KV_BYTES = 4 * KV_BOX;   // 32 KB
+  static constexpr int NB = D * EB / 128;         // 128-byte boxes across a row: 4 (bf16), 2 (E4M3)
+  static constexpr int BOX_COLS = 128 / EB;
+  static constexpr int Q_BOX = 128 * 128;         // 128 rows x 128 B
+  static constexpr int KV_BOX = 64 * 128;         // 64 rows x 128 B
+  static constexpr int Q_BYTES = NB * Q_BOX;      // 64 KB (bf16), 32 KB (E4M3)
+  static constexpr int KV_BYTES = NB * KV_BOX;    // 32 KB (bf16), 16 KB (E4M3)
+  static constexpr int NK_S = D * EB / 32;        // 32-byte K steps of S = Q K^T
+  static constexpr int PV_KEYS = 32 / EB;         // keys per PV MMA step (8 tensor-memory columns of P)
+  static constexpr int NK_PV = BN / PV_KEYS;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;   // 2 stages
   static constexpr int OFF_V = OFF_K + 2 * KV_BYTES;
@@ -49,11 +62,13 @@ struct Fwd256Cfg {
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
-template <bool FP8P, bool COUNT = false>
+template <typename Elem, bool FP8P, bool COUNT = false>
 __global__ void __launch_bounds__(192, 1)
     fa_fwd256_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const Fwd256Args a) {
-  using C = Fwd256Cfg;
+  constexpr int EB = sizeof(Elem);
+  static_assert(EB == 2 || (EB == 1 && FP8P), "bf16 operands, or E4M3 operands with the P-cast");
+  using C = Fwd256Cfg<EB>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ uint64_t bar_q, bar_kf[2], bar_ke[2], bar_vf[2], bar_ve[2], bar_s[2], bar_p[2], bar_pv, bar_o, bar_done;
@@ -75,6 +90,7 @@ __global__ void __launch_bounds__(192, 1)
   const int n_kv = (N + 63) >> 6;
   const int T = a.causal ? min(n_kv, 2 * qt + 2) : n_kv;  // key tiles this Q tile sees
   const bool rev = FP8P && a.kv_order;                       // visit them T-1 .. 0
+  constexpr bool kE4M3 = EB == 1;
 
   if (warp == 5) {
     tmem_alloc(&tmem_base_sh, 512);
@@ -108,7 +124,8 @@ __global__ void __launch_bounds__(192, 1)
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       mbar_arrive_expect_tx(&bar_q, C::Q_BYTES);
-      for (int b = 0; b < 4; ++b) tma_load_3d(smem + C::OFF_Q + b * C::Q_BOX, &tmQ, &bar_q, b * 64, m0, bh);
+      for (int b = 0; b < C::NB; ++b)
+        tma_load_3d(smem + C::OFF_Q + b * C::Q_BOX, &tmQ, &bar_q, b * C::BOX_COLS, m0, bh);
       int t = 0;
       for (; t < T; ++t) {
         const int s = t & 1;
@@ -116,12 +133,14 @@ __global__ void __launch_bounds__(192, 1)
         if (!mbar_wait(&bar_ke[s], ph ^ 1, &abort_sh, 80)) break;
         const int j = rev ? T - 1 - t : t;
         mbar_arrive_expect_tx(&bar_kf[s], C::KV_BYTES);
-        for (int b = 0; b < 4; ++b)
-          tma_load_3d(smem + C::OFF_K + s * C::KV_BYTES + b * C::KV_BOX, &tmK, &bar_kf[s], b * 64, j * 64, bh_kv);
+        for (int b = 0; b < C::NB; ++b)
+          tma_load_3d(smem + C::OFF_K + s * C::KV_BYTES + b * C::KV_BOX, &tmK, &bar_kf[s], b * C::BOX_COLS, j * 64,
+                      bh_kv);
         if (!mbar_wait(&bar_ve[s], ph ^ 1, &abort_sh, 81)) break;
         mbar_arrive_expect_tx(&bar_vf[s], C::KV_BYTES);
-        for (int b = 0; b < 4; ++b)
-          tma_load_3d(smem + C::OFF_V + s * C::KV_BYTES + b * C::KV_BOX, &tmV, &bar_vf[s], b * 64, j * 64, bh_kv);
+        for (int b = 0; b < C::NB; ++b)
+          tma_load_3d(smem + C::OFF_V + s * C::KV_BYTES + b * C::KV_BOX, &tmV, &bar_vf[s], b * C::BOX_COLS, j * 64,
+                      bh_kv);
       }
       mbar_wait_drain(&bar_q, 0, 100000000ull);
       for (int u = max(0, t - 2); u < t; ++u) {
@@ -132,18 +151,23 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp == 5) {
     // ============================ MMA issuer =================================
     if (lane == 0) {
-      constexpr uint32_t id_s = make_idesc(128, 64, kFmtBF16, 0, 0);   // S = Q K^T: N = 64 keys, K = 256
-      constexpr uint32_t id_pv = make_idesc(128, 256, kFmtBF16, 0, 1); // O += P V: N = 256, K = 64 keys
+      constexpr uint32_t fmt = kE4M3 ? kFmtE4M3 : kFmtBF16;
+      constexpr uint32_t id_s = make_idesc(128, 64, fmt, 0, 0);   // S = Q K^T: N = 64 keys, K = 256
+      constexpr uint32_t id_pv = make_idesc(128, 256, fmt, 0, 1); // O += P V: N = 256, K = 64 keys
       const uint32_t q_addr = smem_u32(smem + C::OFF_Q);
       const uint32_t k_addr = smem_u32(smem + C::OFF_K), v_addr = smem_u32(smem + C::OFF_V);
       auto issue_s = [&](int t) {
         const int s = t & 1;
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
+        for (int k = 0; k < C::NK_S; ++k) {
           const uint32_t qa = q_addr + (k >> 2) * C::Q_BOX + (k & 3) * 32;
           const uint32_t ka = k_addr + s * C::KV_BYTES + (k >> 2) * C::KV_BOX + (k & 3) * 32;
-          mma_ss(tmem + C::COL_S + 64 * s, make_sdesc_sw128(qa, 16, 1024), make_sdesc_sw128(ka, 16, 1024), id_s,
-                 k > 0);
+          if constexpr (kE4M3)
+            mma_ss_f8(tmem + C::COL_S + 64 * s, make_sdesc_sw128(qa, 16, 1024), make_sdesc_sw128(ka, 16, 1024), id_s,
+                      k > 0);
+          else
+            mma_ss(tmem + C::COL_S + 64 * s, make_sdesc_sw128(qa, 16, 1024), make_sdesc_sw128(ka, 16, 1024), id_s,
+                   k > 0);
         }
         mma_commit(&bar_s[s]);
         mma_commit(&bar_ke[s]);
@@ -160,12 +184,16 @@ __global__ void __launch_bounds__(192, 1)
         if (!(ok = mbar_wait(&bar_vf[s], ph, &abort_sh, 84))) break;
         if (!(ok = mbar_wait(&bar_p[s], ph, &abort_sh, 85))) break;
         tc_fence_after();
-        // O += P(t) V(t): A = P from TMEM (bf16, 16 keys = 8 columns per step), B = V MN-major
+        // O += P(t) V(t): A = P from TMEM (8 columns per step: 16 bf16 or 32 E4M3
+        // keys), B = V MN-major, K rows 128 B apart
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          mma_ts(tmem + C::COL_O, tmem + C::COL_S + 64 * s + k * 8,
-                 make_sdesc_sw128(v_addr + s * C::KV_BYTES + k * 2048, C::KV_BOX, 1024), id_pv,
-                 (t > 0 || k > 0) ? 1u : 0u);
+        for (int k = 0; k < C::NK_PV; ++k) {
+          const uint64_t bd = make_sdesc_sw128(v_addr + s * C::KV_BYTES + k * C::PV_KEYS * 128, C::KV_BOX, 1024);
+          if constexpr (kE4M3)
+            mma_ts_f8(tmem + C::COL_O, tmem + C::COL_S + 64 * s + k * 8, bd, id_pv, (t > 0 || k > 0) ? 1u : 0u);
+          else
+            mma_ts(tmem + C::COL_O, tmem + C::COL_S + 64 * s + k * 8, bd, id_pv, (t > 0 || k > 0) ? 1u : 0u);
+        }
         mma_commit(&bar_ve[s]);
         mma_commit(&bar_pv);
         if (t + 2 < T) {
@@ -183,7 +211,8 @@ __global__ void __launch_bounds__(192, 1)
     const int r = threadIdx.x;  // row in tile == TMEM lane
     const int row = m0 + r;
     const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;
-    const float c = a.scale_log2;
+    // E4M3 operands: the score factor of key tile j carries sq[query block] sk[key block]
+    const float c_base = kE4M3 ? a.scale_log2 * a.sq[static_cast<size_t>(bh) * a.nqb + qt] : a.scale_log2;
     // with the P-cast the exponent carries log2(S): the exps give S p, l sums S p
     const float lg2S = FP8P ? log2f(a.p_scale) : 0.f;
     float m_run = -INFINITY, l_run = 0.f;
@@ -200,6 +229,7 @@ __global__ void __launch_bounds__(192, 1)
       tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
       tmem_wait_ld();
       const int kbase = j * 64;
+      const float c = kE4M3 ? c_base * a.sk[static_cast<size_t>(bh_kv) * a.nqb + (kbase >> 7)] : c_base;
       if (kbase + 64 > N || (a.causal && kbase + 63 > m0)) {
         const int lim = a.causal ? min(N - 1, row) : N - 1;
 #pragma unroll
@@ -243,8 +273,25 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       float2 rs4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-      uint32_t pk[32];
       uint32_t nz2 = 0;  // COUNT: f16x2 counter of non-zero P' (at most 32 per half)
+      if constexpr (kE4M3) {
+        // P' = E4M3(S p) as the PV MMA's A operand: four codes per column
+        uint32_t pk8[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float2 x01 = ffma2(make_float2(sv[4 * e], sv[4 * e + 1]), c2, nm2);
+          const float2 x23 = ffma2(make_float2(sv[4 * e + 2], sv[4 * e + 3]), c2, nm2);
+          const float2 s01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
+          const float2 s23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
+          rs4[e & 3] = fadd2(rs4[e & 3], fadd2(s01, s23));
+          uint16_t lo, hi;
+          asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(s01.y), "f"(s01.x));
+          asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(s23.y), "f"(s23.x));
+          pk8[e] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+        }
+        tmem_st16(tS, pk8);
+      } else {
+      uint32_t pk[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
         const float2 x = ffma2(make_float2(sv[2 * e], sv[2 * e + 1]), c2, nm2);
@@ -259,6 +306,7 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       tmem_st32(tS, pk);
+      }
       if constexpr (COUNT) {
         if (row < N) {
           const uint32_t nf_tile = f16x2_sum_u32(nz2);
@@ -295,7 +343,8 @@ __global__ void __launch_bounds__(192, 1)
     if (ok) ok = mbar_wait(&bar_o, 0, &abort_sh, 89);
     if (ok) {
       tc_fence_after();
-      const float inv = 1.0f / l_run;
+      // l_run sums S p when P is cast; E4M3 V carries its per-head scale
+      const float inv = (kE4M3 ? a.sv[bh_kv] : 1.0f) / l_run;
       __nv_bfloat16* orow = a.o + (static_cast<size_t>(bh) * N + row) * C::D;
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {

@@ -179,7 +179,7 @@ int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, 
  *  - v, one scale per head, never rotated.
  * Outputs (caller-owned device memory): q8, k8, v8 uint8 [B,H,N,d] E4M3 codes;
  * sq, sk fp32 [B,H,ceil(N/128)] and sv fp32 [B,H] dequantisation scales
- * (block amax / 448, 1 for an all-zero block).  d in {64, 128}. */
+ * (block amax / 448, 1 for an all-zero block).  d in {64, 128, 256}. */
 int fa_fp8_quantize(const void* q, const void* k, const void* v, const float* signs, void* q8, void* k8, void* v8,
                     float* sq, float* sk, float* sv, int B, int H, int N, int d, void* stream);
 
@@ -187,8 +187,9 @@ int fa_fp8_quantize(const void* q, const void* k, const void* v, const float* si
  * the kind::f8f6f4 tensor cores, the online softmax in fp32, P' = E4M3(S_p p)
  * (static scale S_p, key-tile order kv_order as in fa_fwd_fp8p), O += P' v8 on
  * the tensor cores, and O = acc * sv / (S_p * l) -> bf16 [B,H,N,d]; lse fp32
- * [B,H,N] of the quantised scores.  d in {64, 128} (64-byte E4M3 rows at d = 64
- * are staged with the 64-byte swizzle). */
+ * [B,H,N] of the quantised scores.  d in {64, 128, 256} (64-byte E4M3 rows at
+ * d = 64 are staged with the 64-byte swizzle; at d = 256 the key tiles are 64
+ * keys, so the running max of the P-cast moves once per 64 keys). */
 int fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* sq, const float* sk, const float* sv,
                void* o, float* lse, int B, int H, int N, int d, int causal, float scale, float S, int kv_order,
                void* stream);

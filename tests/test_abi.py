@@ -117,15 +117,16 @@ def test_head_dim_256_is_admitted_where_declared(lib):
     assert lib.fa_decode(good, good, good, good, good, 1, 4, 1, 64, 96, 0.1, good, 1 << 30, None) == 2
     assert lib.fa_decode(good, good, good, good, good, 1, 32, 1, 64, 256, 0.1, good, 1 << 30, None) == 2  # g > 16
     lib.fa_fwd_fp8.argtypes = [vp] * 3 + [vp] * 3 + [vp, vp] + [ci] * 5 + [cf, cf, ci, vp]
-    assert lib.fa_fwd_fp8(*([good] * 8), 1, 1, 64, 256, 1, 0.1, 256.0, 0, None) == 2      # FP8 takes d = 64, 128
+    assert lib.fa_fwd_fp8(*([good] * 8), 1, 1, 64, 96, 1, 0.1, 256.0, 0, None) == 2       # FP8 takes d = 64, 128, 256
     lib.fa_fwd_fp8_gqa.argtypes = [vp] * 8 + [ci] * 6 + [cf, cf, ci, vp]
     assert lib.fa_fwd_fp8_gqa(*([good] * 8), 1, 6, 4, 64, 128, 1, 0.1, 256.0, 0, None) == 1  # H % H_kv != 0
     assert lib.fa_fwd_fp8_gqa(*([good] * 8), 1, 8, 0, 64, 128, 1, 0.1, 256.0, 0, None) == 1  # H_kv = 0
-    assert lib.fa_fwd_fp8_gqa(*([good] * 8), 1, 8, 2, 64, 256, 1, 0.1, 256.0, 0, None) == 2  # d in {64, 128}
+    assert lib.fa_fwd_fp8_gqa(*([good] * 8), 1, 8, 2, 64, 96, 1, 0.1, 256.0, 0, None) == 2   # d in {64, 128, 256}
     assert lib.fa_fwd_fp8_gqa(*([good] * 8), 1, 8, 2, 64, 128, 1, 0.1, 256.0, 2, None) == 1  # bad kv_order
+    assert lib.fa_fwd_fp8_gqa(*([good] * 8), 1, 8, 2, 64, 256, 1, 0.1, 256.0, 2, None) == 1  # d = 256 admitted
     lib.fa_fp8_quantize_gqa.argtypes = [vp] * 10 + [ci] * 5 + [vp]
     assert lib.fa_fp8_quantize_gqa(*([good] * 10), 1, 6, 4, 64, 128, None) == 1             # H % H_kv != 0
-    assert lib.fa_fp8_quantize_gqa(*([good] * 10), 1, 8, 2, 64, 256, None) == 2             # d in {64, 128}
+    assert lib.fa_fp8_quantize_gqa(*([good] * 10), 1, 8, 2, 64, 96, None) == 2              # d in {64, 128, 256}
 
 
 def test_size_limits_and_lse_alignment(lib):

@@ -43,9 +43,9 @@ def _one_step_apart(got, ref):
     return float((diff > 1e-9 * np.abs(ref)).mean()), bool((diff <= step * 1.0001).all())
 
 
-@pytest.mark.parametrize("rotate", [False, True])
-def test_quantiser_matches_oracle(rotate):
-    B, H, N, d = 1, 2, 300, 128
+@pytest.mark.parametrize("rotate,d", [(False, 128), (True, 128), (True, 64), (True, 256)])
+def test_quantiser_matches_oracle(rotate, d):
+    B, H, N = 1, 2, 300
     x = synth.make_outlier_inputs(B, H, N, d, seed=61)
     signs = synth.random_signs(d, seed=62) if rotate else None
     q8, k8, v8, sq, sk, sv = _gpu_quant(x, signs)
@@ -118,6 +118,27 @@ def test_fp8_forward_head_dim_64(B, H, N, causal, rotate, order):
     signs = synth.random_signs(d, seed=91) if rotate else None
     o, lse = _fp8_forward(x, signs, causal, order)
     o_em, lse_em = _oracle_fp8(x, signs, causal, order)
+    o_ex, _ = oracle.attn_fwd(x["q"], x["k"], x["v"], causal, 1 / math.sqrt(d))
+    assert np.abs(lse - lse_em).max() <= 2e-3
+    mse, mse_em = ((o - o_ex) ** 2).mean(), ((o_em - o_ex) ** 2).mean()
+    assert abs(mse - mse_em) <= 0.1 * mse_em
+    diff = np.abs(o - o_em)
+    assert (diff > 2e-2).mean() <= 1e-3 and diff.max() <= 0.15
+
+
+@pytest.mark.parametrize("B,H,N,causal,rotate,order", [(1, 2, 700, False, True, 0), (1, 1, 333, True, True, 1),
+                                                        (1, 2, 200, True, False, 0)])
+def test_fp8_forward_head_dim_256(B, H, N, causal, rotate, order):
+    """d = 256: the 64-key-tile kernel on E4M3 operands (two 128-byte boxes per
+    row); the running max moves once per 64 keys, so the emulation takes B_c = 64."""
+    d = 256
+    x = synth.make_inputs(B, H, N, d, "bf16", seed=95 + N)
+    signs = synth.random_signs(d, seed=96) if rotate else None
+    o, lse = _fp8_forward(x, signs, causal, order)
+    qq, _ = oracle.fp8_quantize(x["q"], signs)
+    kq, _ = oracle.fp8_quantize(x["k"], signs)
+    vq, _ = oracle.fp8_quantize(x["v"], None, block_rows=N)
+    o_em, lse_em = oracle.attn_fwd_fp8p(qq, kq, vq, causal, 1 / math.sqrt(d), 256.0, order, 64)[:2]
     o_ex, _ = oracle.attn_fwd(x["q"], x["k"], x["v"], causal, 1 / math.sqrt(d))
     assert np.abs(lse - lse_em).max() <= 2e-3
     mse, mse_em = ((o - o_ex) ** 2).mean(), ((o_em - o_ex) ** 2).mean()
