@@ -14,10 +14,11 @@
  *    device arrays (the (batch, heads, seq, head_dim) layout of the pages'
  *    framework example); lse is a contiguous [B, H, N] float32 device array.
  *    LSE is the natural-log logsumexp of the scaled scores of each query row.
- *  - Sizes: B >= 1, H >= 1, N >= 1, d in {64, 128} (fa_fwd, fa_fwd_gqa, fa_bwd,
- *    fa_bwd_gqa, fa_bwd_noalloc and fa_decode also take d = 256, "FlashAttention
- *    (IT)", "FlashAttention-2 (2023)").  Limits of the launches: N <= 2^30,
- *    B*H < 2^31, B*H*ceil(N/128) < 2^31 and B*H*N*d < 2^40; element offsets
+ *  - Sizes: B >= 1, H >= 1, N >= 1, d in {64, 128}; every entry point but
+ *    fa_fwd_f32 (d = 64 only) also takes d = 256 ("FlashAttention (IT)",
+ *    "FlashAttention-2 (2023)").  Limits of the launches: N <= 2^30,
+ *    B*H < 2^31, B*H*ceil(N/128) < 2^31 (twice that for the d = 256 backward,
+ *    which runs two CTAs per key tile) and B*H*N*d < 2^40; element offsets
  *    are 64-bit, so any size that fits in device memory within these is taken.
  *  - scale: the softmax scale (usually 1/sqrt(d)); finite and > 0.
  *  - causal != 0: query i attends to keys j <= i (square, top-left aligned);
@@ -54,8 +55,9 @@ typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, bad scale/S/kv_order */
   FA_ERR_UNSUPPORTED = 2, /* a head dim the entry point does not take (64 and 128
-                             everywhere; 256 only where its comment says so), sizes
-                             over the limits above, B*H_kv > 65535 (fa_decode) or
+                             everywhere but fa_fwd_f32, which takes 64; 256 where
+                             the entry point's comment says so), sizes over the
+                             limits above, B*H_kv > 65535 (fa_decode) or
                              B*H > 65535 (fa_fp8_quantize), more than 16 query heads
                              per key/value head (fa_decode), or a workspace larger
                              than FA_BWD_NOALLOC_MAX_BYTES (fa_bwd_noalloc) */
