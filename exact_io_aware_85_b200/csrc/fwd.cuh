@@ -417,6 +417,10 @@ __global__ void __launch_bounds__(384, 1)
     // With a P-cast (FP8P or E4M3 operands) the exponent carries log2(S): the
     // exps give q = S p directly, l sums q, and the epilogue divides by it.
     constexpr bool kCast = FP8P || C::EB == 1;
+    // With the flush counting (more ALU work per key) 1 of every 8 key pairs on
+    // the FMA pipe pays: sink workload 1013 -> 1026 TFLOP/s; without it (1146 ->
+    // 1103) and in the plain bf16 forward at d = 128 (1112 -> 1084) it does not.
+    constexpr int kExpPoly = COUNT ? 1 : C::EXP_POLY;
     const float lg2S = kCast ? log2f(a.p_scale) : 0.f;
     float m_run = -INFINITY, l_run = 0.f;
     uint32_t nf_sink = 0, nf_non = 0;  // COUNT: P' that did not flush, per key class
@@ -532,7 +536,7 @@ __global__ void __launch_bounds__(384, 1)
             for (int e = 0; e < PC; ++e) {
               const float2 x = ffma2(make_float2(sv[h * 2 * PC + 2 * e], sv[h * 2 * PC + 2 * e + 1]), c2, nm2);
               float p0, p1;  // S p with FP8P, p otherwise
-              if ((e & 7) < C::EXP_POLY) {
+              if ((e & 7) < kExpPoly) {
                 const float2 pp = exp2_fma2(x);
                 p0 = pp.x;
                 p1 = pp.y;
