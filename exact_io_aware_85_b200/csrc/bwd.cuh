@@ -136,6 +136,10 @@ struct BwdCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
+// dst[0..1] += (lo, hi) (fp32) as one 8-byte reduction in the L2
+__device__ __forceinline__ void red_add_v2(float* dst, float lo, float hi) {
+  asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(dst), "f"(lo), "f"(hi) : "memory");
+}
 // dst[0..3] += v[0..3] (fp32) as one 16-byte reduction in the L2
 __device__ __forceinline__ void red_add_v4(float* dst, const uint32_t* v) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(__uint_as_float(v[0])),
@@ -741,9 +745,22 @@ __global__ void __launch_bounds__(512, 1)
       if (fill) mbar_arrive(bar_dp_init);
       if (t >= 1) {
         const int i = step_tile(t - 1), hq = step_head(t - 1);
-        float* dst = a.dq_acc + (static_cast<size_t>(hq) * a.Npad + static_cast<size_t>(i) * 128) * C::D + c;
+        // lane pairs (c even, c + 1): the even lane adds columns c, c + 1 of the
+        // even queries, the odd lane those of the odd queries, 8 bytes at a time
+        // (half the reduction instructions of one 4-byte add per query; training
+        // step 817 -> 833 TFLOP/s)
+        const int c0 = c & ~1;
+        float* dst = a.dq_acc + (static_cast<size_t>(hq) * a.Npad + static_cast<size_t>(i) * 128) * C::D + c0;
+        const bool odd = (c & 1) != 0;
 #pragma unroll
-        for (int q = 0; q < 128; ++q) atomicAdd(dst + static_cast<size_t>(q) * C::D, __uint_as_float(v[q]));
+        for (int q2 = 0; q2 < 64; ++q2) {
+          const float give = __uint_as_float(odd ? v[2 * q2] : v[2 * q2 + 1]);
+          const float got = __shfl_xor_sync(0xffffffffu, give, 1);
+          const int q = 2 * q2 + (odd ? 1 : 0);
+          const float mine = __uint_as_float(odd ? v[2 * q2 + 1] : v[2 * q2]);
+          const float lo = odd ? got : mine, hi = odd ? mine : got;
+          red_add_v2(dst + static_cast<size_t>(q) * C::D, lo, hi);
+        }
       }
     }
     tc_fence_before();
