@@ -63,6 +63,20 @@ signs = torch.from_numpy(synth.random_signs(128, seed=1)).cuda()
 fa.fa_fp8_quantize(q, k, v, signs, q8, k8, v8, sq, sk, sv)
 fa.fa_fwd_fp8(q8, k8, v8, sq, sk, sv, o, lse, True, 1 / math.sqrt(128), 256.0, 0)
 torch.cuda.synchronize(); out["fp8"] = (o.float().cpu().numpy(),)
+for dd, nn in ((64, 200), (256, 150)):  # 64-byte E4M3 rows; the 64-key-tile kernel
+    x = synth.make_inputs(1, 2, nn, dd, "bf16", seed=dd + 3)
+    q, k, v = (t(x[n]) for n in ("q", "k", "v"))
+    o = torch.empty_like(q); lse = torch.empty((1, 2, nn), device="cuda")
+    nb = (nn + 127) // 128
+    q8, k8, v8 = (torch.empty(q.shape, dtype=torch.uint8, device="cuda") for _ in range(3))
+    sq, sk = (torch.empty((1, 2, nb), device="cuda") for _ in range(2)); sv = torch.empty((1, 2), device="cuda")
+    fa.fa_fp8_quantize(q, k, v, None, q8, k8, v8, sq, sk, sv)
+    fa.fa_fwd_fp8(q8, k8, v8, sq, sk, sv, o, lse, True, 1 / math.sqrt(dd), 256.0, 1)
+    torch.cuda.synchronize(); out[f"fp8_{dd}"] = (o.float().cpu().numpy(),)
+    if dd == 256:
+        st = torch.zeros(4, dtype=torch.int64, device="cuda")
+        fa.fa_fwd_fp8p(q, k, v, o, lse, True, 1 / math.sqrt(dd), 256.0, 1, st, 4)
+        torch.cuda.synchronize(); out["fp8p_256"] = (o.float().cpu().numpy(), st.cpu().numpy())
 xd = synth.make_inputs(2, 4, 1000, 128, "bf16", seed=7)
 qd = t(xd["q"][:, :, 0]); kd, vd = t(xd["k"][:, :2]), t(xd["v"][:, :2])
 od = torch.empty_like(qd); lsed = torch.empty((2, 4), device="cuda")
