@@ -187,7 +187,7 @@ def measure_fp8_peak(n: int = 8192, reps: int = 10):
     return 2.0 * n ** 3 / (best * 1e-3) / 1e12
 
 
-def cpu_baseline(w: synth.Workload, target_s: float = 12.0):
+def cpu_baseline(w: synth.Workload, target_s: float = 14.0):
     """The fp64 oracle on the host cores over a bounded sample of query rows of
     the same workload; TFLOP/s of useful attention work."""
     import oracle
@@ -205,9 +205,9 @@ def cpu_baseline(w: synth.Workload, target_s: float = 12.0):
         t0 = time.perf_counter()
         oracle.attn_fwd_rows(x["q"], x["k"], x["v"], rows, w.causal, w.scale)
         dt = time.perf_counter() - t0
-        if dt >= 0.5 * target_s or n >= 400000:
+        if dt >= 0.7 * target_s or n >= 1000000:
             break
-        n = int(min(400000, n * max(2.0, 0.9 * target_s / max(dt, 1e-3))))
+        n = int(min(1000000, n * max(2.0, 0.9 * target_s / max(dt, 1e-3))))
     rate = flops(rows) / dt
     return {"value": rate / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
             "sample": f"{n} random query rows of one head of the {w.name} workload (N={w.N}, d={w.d}, "
