@@ -598,7 +598,7 @@ int fa_fp8_quantize_gqa(const void* q, const void* k, const void* v, const float
     fa::fa_fp8_qk_quant_kernel<64><<<grid, 128, 0, s>>>(a);
     fa::fa_fp8_v_quant_kernel<64><<<static_cast<unsigned>((nvec + 255) / 256), 256, 0, s>>>(a, nvec);
   } else if (d == 256) {
-    fa::fa_fp8_qk_quant_kernel<256><<<grid, 128, 0, s>>>(a);
+    fa::fa_fp8_qk_quant256_kernel<<<grid, 256, 0, s>>>(a);
     fa::fa_fp8_v_quant_kernel<256><<<static_cast<unsigned>((nvec + 255) / 256), 256, 0, s>>>(a, nvec);
   } else {
     fa::fa_fp8_qk_quant_kernel<128><<<grid, 128, 0, s>>>(a);

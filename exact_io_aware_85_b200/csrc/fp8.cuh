@@ -136,6 +136,86 @@ __global__ void __launch_bounds__(128) fa_fp8_qk_quant_kernel(const Fp8QuantArgs
   }
 }
 
+// d = 256: two lanes per row (lanes l and l ^ 16 of a warp hold columns
+// [0, 128) and [128, 256)), so that no thread keeps a whole row in registers.
+// The Hadamard transform's stages h = 1 .. 64 stay inside each half; its last
+// stage pairs column i with i + 128, the two lanes of the row: a shuffle
+// butterfly.  Otherwise as fa_fp8_qk_quant_kernel (one CTA = 128 rows).
+__global__ void __launch_bounds__(256) fa_fp8_qk_quant256_kernel(const Fp8QuantArgs a) {
+  constexpr int D = 256, HD = 128;
+  __shared__ float red[8];
+  const int blk = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;  // 0 Q, 1 K, 2 V maxima
+  // grid.y covers the larger head count; the whole CTA leaves before any barrier
+  if (bh >= (which == 0 ? a.BH : a.BH_kv)) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int half = lane >> 4;
+  const int row = blk * 128 + warp * 16 + (lane & 15);
+  const bool live = row < a.N;
+  const __nv_bfloat16* src = which == 0 ? a.q : (which == 1 ? a.k : a.v);
+  float x[HD];
+  if (live) {
+    const uint4* p = reinterpret_cast<const uint4*>(src + (static_cast<size_t>(bh) * a.N + row) * D + half * HD);
+#pragma unroll
+    for (int c = 0; c < HD / 8; ++c) {
+      const uint4 w = p[c];
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(h[e]);
+        x[8 * c + 2 * e] = f.x;
+        x[8 * c + 2 * e + 1] = f.y;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < HD; ++c) x[c] = 0.f;
+  }
+  if (which < 2 && a.signs != nullptr) {
+#pragma unroll
+    for (int c = 0; c < HD; ++c) x[c] *= a.signs[half * HD + c];
+    fwht_row<HD>(x);
+#pragma unroll
+    for (int c = 0; c < HD; ++c) {
+      const float o = __shfl_xor_sync(0xffffffffu, x[c], 16);
+      x[c] = half ? o - x[c] : x[c] + o;  // (a + b, a - b) over the lanes (lo, hi)
+    }
+    const float norm = rsqrtf(static_cast<float>(D));
+#pragma unroll
+    for (int c = 0; c < HD; ++c) x[c] *= norm;
+  }
+  float am = 0.f;
+#pragma unroll
+  for (int c = 0; c < HD; ++c) am = fmaxf(am, fabsf(x[c]));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
+  if (lane == 0) red[warp] = am;
+  __syncthreads();
+  float amax = red[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) amax = fmaxf(amax, red[w]);
+  if (which == 2) {
+    if (threadIdx.x == 0) atomicMax(reinterpret_cast<int*>(a.sv) + bh, __float_as_int(amax));
+    return;
+  }
+  const float scale = amax > 0.f ? amax / 448.f : 1.f;
+  if (threadIdx.x == 0) (which == 0 ? a.sq : a.sk)[static_cast<size_t>(bh) * a.nblk + blk] = scale;
+  if (!live) return;
+  uint8_t* dst = (which == 0 ? a.q8 : a.k8) + (static_cast<size_t>(bh) * a.N + row) * D + half * HD;
+#pragma unroll
+  for (int c = 0; c < HD / 16; ++c) {
+    uint4 w;
+    w.x = e4m3x4(__fdiv_rn(x[16 * c + 0], scale), __fdiv_rn(x[16 * c + 1], scale), __fdiv_rn(x[16 * c + 2], scale),
+                 __fdiv_rn(x[16 * c + 3], scale));
+    w.y = e4m3x4(__fdiv_rn(x[16 * c + 4], scale), __fdiv_rn(x[16 * c + 5], scale), __fdiv_rn(x[16 * c + 6], scale),
+                 __fdiv_rn(x[16 * c + 7], scale));
+    w.z = e4m3x4(__fdiv_rn(x[16 * c + 8], scale), __fdiv_rn(x[16 * c + 9], scale),
+                 __fdiv_rn(x[16 * c + 10], scale), __fdiv_rn(x[16 * c + 11], scale));
+    w.w = e4m3x4(__fdiv_rn(x[16 * c + 12], scale), __fdiv_rn(x[16 * c + 13], scale),
+                 __fdiv_rn(x[16 * c + 14], scale), __fdiv_rn(x[16 * c + 15], scale));
+    reinterpret_cast<uint4*>(dst)[c] = w;
+  }
+}
+
 // Clears the per-head V maxima before fa_fp8_qk_quant_kernel accumulates them.
 __global__ void fa_fp8_v_clear_kernel(float* sv, int BH) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
