@@ -38,10 +38,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # that kernel (dram__bytes_read.sum + dram__bytes_write.sum); reported only while
 # the kernel sources still hash to the values they were measured with.
 TRAFFIC = {
-    "prefill": {"bytes": 808655104 + 253243648, "src": ("fwd.cuh", "sm100.cuh"),
-                "sha1": "81d40e2f1bfad2e67608ed9efe314374c6d0e79f"},
-    "decode": {"bytes": 1073833728 + 3366144, "src": ("decode.cuh", "sm100.cuh"),
-               "sha1": "548786c61733f222f70418c2560262e3d380d330"},
+    "prefill": {"bytes": 807555328 + 253336832, "src": ("fwd.cuh", "sm100.cuh"),
+                "sha1": "d17a89c792c0f38b6388ce3907e811ffde3c2927"},
+    "decode": {"bytes": 1073828608 + 3488256, "src": ("decode.cuh", "sm100.cuh"),
+               "sha1": "725bc8cae726ee0b4c4ac46b4da2a68672b5a5e5"},
 }
 
 

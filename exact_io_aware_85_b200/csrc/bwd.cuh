@@ -140,12 +140,6 @@ struct BwdCfg {
 __device__ __forceinline__ void red_add_v2(float* dst, float lo, float hi) {
   asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(dst), "f"(lo), "f"(hi) : "memory");
 }
-// dst[0..3] += v[0..3] (fp32) as one 16-byte reduction in the L2
-__device__ __forceinline__ void red_add_v4(float* dst, const uint32_t* v) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(__uint_as_float(v[0])),
-               "f"(__uint_as_float(v[1])), "f"(__uint_as_float(v[2])), "f"(__uint_as_float(v[3]))
-               : "memory");
-}
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(

@@ -157,20 +157,7 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void*
       "r"(smem_u32(smem_src)), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
-// shared -> global tiled bulk reduction: the global tile += the shared tile
-// (element type of the tensor map), tracked like the stores
-__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, const void* smem_src, int x, int y, int z) {
-  if (!FA_CHECK((smem_u32(smem_src) & 127u) == 0 && x >= 0 && (x & 7) == 0 && y >= 0 && z >= 0, 202)) return;
-  asm volatile(
-      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
-          reinterpret_cast<uint64_t>(map)),
-      "r"(smem_u32(smem_src)), "r"(x), "r"(y), "r"(z)
-      : "memory");
-}
 __device__ __forceinline__ void tma_store_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// wait until every committed bulk store/reduction of this thread has finished
-// reading its shared-memory source (the global writes may still be in flight)
-__device__ __forceinline__ void tma_store_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // wait until every committed bulk store of this thread has completed
 __device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
@@ -224,22 +211,6 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t peer_dst, const void*
                    peer_dst),
                "r"(smem_u32(src)), "r"(bytes), "r"(peer_bar)
                : "memory");
-}
-// 16 bytes into shared memory of a CTA of the cluster (a shared::cluster address)
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint4 v) {
-  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
-               "r"(v.w)
-               : "memory");
-}
-// make this thread's generic-proxy writes to cluster shared memory visible to
-// the async proxy (the peer's tensor-core reads of them)
-__device__ __forceinline__ void fence_proxy_async_cluster() {
-  asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
-}
-// one arrival on a barrier of a CTA of the cluster, releasing this thread's
-// earlier writes at cluster scope
-__device__ __forceinline__ void mbar_arrive_peer(uint32_t peer_bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(peer_bar) : "memory");
 }
 // Bounded wait as mbar_wait, acquiring at cluster scope: for barriers that the
 // peer CTA arrives on.
